@@ -1,0 +1,413 @@
+"""Benchmark of the POET-X layer hot path on B200: forward + backward of the
+Llama-8B decoder block's seven linears (q, k, v, o, gate, up, down; b = 256,
+16384 tokens per GPU), CNP build and CNP backward included, merge excluded.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl poetx|reference]
+
+One step = for every linear: build G_R, G_P from the packed triangles, the
+forward (saving Y), then the backward (dx, dqR, dqP); with N > 1 ranks the
+packed gradients of all linears are summed across ranks (NCCL all-reduce, the
+data-parallel exchange).  Each rank processes its own 16384 tokens (weak
+scaling).  Inputs are synthetic (seeded normal activations / gradients,
+N(0, 0.02^2) weights, N(0, 0.01^2) triangles, seeded permutations), drawn on
+the device; every tensor of the working set is larger than L2.
+
+--impl reference times the float64 CPU oracle (oracle/) on the host cores on
+a bounded token sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import poetx_inputs as pi  # noqa: E402
+
+METRIC = "POET-X layer fwd+bwd tokens/s (Llama-8B shapes, b=256); % bf16 tensor peak"
+WORKLOAD = "block8b"
+# DRAM bytes per launch of the dominant kernel (w0_gemm) from an ncu capture;
+# None until a capture of the current kernel exists.
+W0_GEMM_TRAFFIC_BYTES = None
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def config_block(cfg: pi.Config, n_gpus: int) -> dict:
+    return {"workload": f"{cfg.name}: {cfg.description}",
+            "linears": [f"{nm} {m}x{n}" for nm, m, n in cfg.layers],
+            "tokens_per_gpu": cfg.T, "global_batch": cfg.T * n_gpus, "seq_len": 2048, "b": cfg.b,
+            "parallelism": f"dp{n_gpus}",
+            "l2": "no flush: every input and intermediate is larger than the 126 MB L2"}
+
+
+# ---------------------------------------------------------------- distributed helpers
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), int(
+        os.environ.get("LOCAL_RANK", "0"))
+
+
+def reduce_max(value: float, device) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def allreduce_grads(flat) -> None:
+    """Sum the packed gradients of every linear across data-parallel ranks."""
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(flat, op=dist.ReduceOp.SUM)
+
+
+def barrier(device) -> None:
+    import torch
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier(device_ids=[device.index] if device.type == "cuda" else None)
+    if device.type == "cuda":
+        torch.cuda.synchronize(device)
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", self.gpu_id], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=5)
+        sm, smax, power, reasons = [], [], [], set()
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for name, v in zip(self.NAMES, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power) if power else None}
+
+
+# ---------------------------------------------------------------- POET-X arm
+def build_block(cfg: pi.Config, device, rank: int):
+    import torch
+    import orthogonal_equivalence_b200 as px
+    layers = []
+    for li, (name, m, n) in enumerate(cfg.layers):
+        g = torch.Generator(device=device)
+        g.manual_seed(pi.seed_of(cfg, li, "W0"))
+        W0lin = (torch.randn((n, m), generator=g, device=device, dtype=torch.float32) * 0.02).to(torch.bfloat16)
+        gc = torch.Generator()
+        gc.manual_seed(pi.seed_of(cfg, li, "permR"))
+        permR = torch.randperm(m, generator=gc).to(torch.int32)
+        gc.manual_seed(pi.seed_of(cfg, li, "permP"))
+        permP = torch.randperm(n, generator=gc).to(torch.int32)
+        tri = cfg.b * (cfg.b - 1) // 2
+        g.manual_seed(pi.seed_of(cfg, li, "qR"))
+        qR = torch.randn((m // cfg.b, tri), generator=g, device=device) * cfg.sigma_q
+        g.manual_seed(pi.seed_of(cfg, li, "qP"))
+        qP = torch.randn((n // cfg.b, tri), generator=g, device=device) * cfg.sigma_q
+        L = px.PoetxLinear(m, n, cfg.b, px.POETX_BF16, device=device)
+        L.load(W0lin, permR, permP, qR, qP)
+        del W0lin
+        # per-rank data (each data-parallel rank sees its own tokens)
+        g.manual_seed(pi.seed_of(cfg, li, "x") + 7919 * rank)
+        x = torch.randn((cfg.T, m), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+        g.manual_seed(pi.seed_of(cfg, li, "dz") + 7919 * rank)
+        dz = torch.randn((cfg.T, n), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+        layers.append({"L": L, "x": x, "dz": dz, "m": m, "n": n})
+    # outputs and saved activations, allocated once
+    nq = sum(l["L"].qR.numel() + l["L"].qP.numel() for l in layers)
+    flat = torch.zeros(nq, dtype=torch.float32, device=device)
+    off = 0
+    for l in layers:
+        L = l["L"]
+        l["z"] = torch.empty((cfg.T, l["n"]), dtype=torch.bfloat16, device=device)
+        l["y"] = torch.empty((cfg.T, l["n"]), dtype=torch.bfloat16, device=device)
+        l["dx"] = torch.empty((cfg.T, l["m"]), dtype=torch.bfloat16, device=device)
+        l["dqR"] = flat[off:off + L.qR.numel()].view_as(L.qR)
+        off += L.qR.numel()
+        l["dqP"] = flat[off:off + L.qP.numel()].view_as(L.qP)
+        off += L.qP.numel()
+    return layers, flat
+
+
+def run_step(layers, flat) -> None:
+    for l in layers:
+        L = l["L"]
+        L.build()
+        L.forward(l["x"], z=l["z"], y=l["y"])
+    for l in reversed(layers):
+        L = l["L"]
+        L.backward(l["x"], l["y"], l["dz"], dx=l["dx"], dqR=l["dqR"], dqP=l["dqP"])
+    allreduce_grads(flat)
+
+
+def bench_poetx(args, cfg: pi.Config) -> dict:
+    import torch
+    import torch.distributed as dist
+    import orthogonal_equivalence_b200 as px
+    from orthogonal_equivalence_b200 import build as pbuild
+
+    rank, world, local = dist_env()
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if rank == 0:
+        pbuild.build()
+    if world > 1:
+        dist.barrier(device_ids=[local])
+    px.lib()
+
+    layers, flat = build_block(cfg, device, rank)
+    torch.cuda.synchronize(device)
+    for _ in range(args.warmup):
+        run_step(layers, flat)
+    barrier(device)
+
+    props = torch.cuda.get_device_properties(device)
+    uuid = getattr(props, "uuid", None)
+    sampler = ClockSampler(f"GPU-{uuid}" if uuid else str(local))
+    sampler.start()
+    time.sleep(0.3)
+    stream = torch.cuda.current_stream(device)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(device)
+    px.poetx_profile_begin()
+    start.record(stream)
+    for _ in range(args.steps):
+        run_step(layers, flat)
+    end.record(stream)
+    torch.cuda.synchronize(device)
+    stages = px.poetx_profile_end()
+    barrier(device)
+    clocks = sampler.stop()
+    ms_local = start.elapsed_time(end)
+    ms_total = reduce_max(ms_local, device)
+
+    # end to end through the public API: pinned host inputs in, gradients out
+    e2e = None
+    if not args.no_e2e:
+        host_x = [l["x"].cpu().pin_memory() for l in layers]
+        host_dz = [l["dz"].cpu().pin_memory() for l in layers]
+        host_dq = torch.empty(flat.numel(), dtype=torch.float32).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host_x + host_dz)
+        d2h = host_dq.numel() * 4
+        e_steps = max(1, min(args.steps, 5))
+
+        def e2e_step():
+            for l, hx, hdz in zip(layers, host_x, host_dz):
+                l["x"].copy_(hx, non_blocking=True)
+                l["dz"].copy_(hdz, non_blocking=True)
+            run_step(layers, flat)
+            host_dq.copy_(flat, non_blocking=True)
+
+        e2e_step()
+        barrier(device)
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record(stream)
+        for _ in range(e_steps):
+            e2e_step()
+        e2.record(stream)
+        torch.cuda.synchronize(device)
+        e_ms = reduce_max(s2.elapsed_time(e2), device)
+        e2e = {"value": world * cfg.T * e_steps / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "steps": e_steps}
+    device_error = px.poetx_device_error()
+
+    peaks, peak_src = measured_peaks()
+    ms_step = ms_total / args.steps
+    flops_step = cfg.flops_per_step()
+    w0_ms, w0_launches = stages["w0_gemm"]
+    w0_flops = cfg.gemm_flops_per_step() * args.steps  # 2Tmn forward + 2Tmn backward per linear
+    peak_sus = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    achieved = w0_flops / (w0_ms / 1e3) / 1e12 if w0_ms > 0 else None
+    total_launches = int(sum(c for _, c in stages.values()))
+    res = {
+        "metric": METRIC,
+        "value": world * cfg.T * args.steps / (ms_total / 1e3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded normal activations and gradients; random-init N(0,0.02^2) weights)",
+        "config": config_block(cfg, world),
+        "tflops_per_gpu": flops_step / (ms_step / 1e3) / 1e12,
+        "pct_bf16_peak": 100.0 * flops_step / (ms_step / 1e3) / 1e12 / peak_sus,
+        "roofline": {"kernel": "w0_gemm", "bound": "tensor", "achieved": achieved,
+                     "peak": peak_sus, "unit": "TFLOP/s",
+                     "frac": (achieved / peak_sus) if achieved else None,
+                     "traffic": W0_GEMM_TRAFFIC_BYTES,
+                     "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)",
+                     "launches": w0_launches,
+                     "algorithmic_flops_per_launch": 2 * sum(cfg.T * m * n for _, m, n in cfg.layers) / len(cfg.layers),
+                     "note": "achieved = algorithmic 2*T*m*n per launch / mean CUDA-event launch time, "
+                             "forward (Y = U W~) and backward (dU = dY W~^T) launches of all 7 linears"},
+        "stages_ms_per_step": {k: v[0] / args.steps for k, v in stages.items()},
+        "gpu_launches": total_launches,
+        "clocks": clocks,
+        "e2e": e2e,
+        "device_error": device_error,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(cfg, args.cpu_tokens)
+    for l in layers:
+        del l["L"]
+    if world > 1:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    return res if rank == 0 else None
+
+
+# ---------------------------------------------------------------- oracle (CPU) arm
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 0) for d in threadpool_info() if d.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_step(cfg: pi.Config, inputs) -> None:
+    import oracle
+    for inp in inputs:
+        W0 = inp.W0lin64.T
+        GR = oracle.cnp_blocks(inp.qR, inp.b)
+        GP = oracle.cnp_blocks(inp.qP, inp.b)
+        oracle.forward(inp.x64, W0, inp.permR, GR, inp.permP, GP)
+        oracle.layer_backward(inp.x64, W0, inp.permR, inp.qR, inp.permP, inp.qP, inp.b, inp.dz64)
+
+
+def oracle_inputs(cfg: pi.Config, tokens: int):
+    return [pi.layer_inputs(cfg, li, T=tokens) for li in range(len(cfg.layers))]
+
+
+def cpu_baseline(cfg: pi.Config, tokens: int) -> dict:
+    inputs = oracle_inputs(cfg, tokens)
+    t0 = time.perf_counter()
+    oracle_step(cfg, inputs)
+    dt = time.perf_counter() - t0
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{tokens} of {cfg.T} tokens through all {len(cfg.layers)} linears (forward, backward, "
+                      f"CNP build and backward, float64), one step, {dt:.1f} s"}
+
+
+def bench_reference(args, cfg: pi.Config) -> dict:
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return None
+    tokens = args.ref_tokens
+    inputs = oracle_inputs(cfg, tokens)
+    for _ in range(args.warmup):
+        oracle_step(cfg, inputs)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(cfg, inputs)
+    dt = time.perf_counter() - t0
+    value = tokens * args.steps / dt
+    sample = (f"{tokens} of {cfg.T} tokens per step through all {len(cfg.layers)} linears (forward, backward, "
+              f"CNP build and backward, float64)")
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded, poetx_inputs recipe)", "config": config_block(cfg, world),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["poetx", "reference"], default="poetx")
+    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(pi.CONFIGS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-tokens", type=int, default=512, help="token sample of the CPU-baseline leg")
+    ap.add_argument("--ref-tokens", type=int, default=64, help="token sample per step of --impl reference")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    cfg = pi.CONFIGS[args.workload]
+    res = bench_reference(args, cfg) if args.impl == "reference" else bench_poetx(args, cfg)
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,169 @@
+/*
+ * poetx.h - C ABI of the POET-X orthogonal-equivalence linear layer for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The layer (POET-X write-up, zhichai.net, "POET-X：单卡H100训练130亿参数模型",
+ * sections 1-3):
+ *   z = P^T (W0^T (R^T x))                       section 1, input-centric form
+ *   R = Psi_R^T Diag(G_R1..G_R,m/b) Psi_R        section 2, block-stochastic R
+ *   P = Psi_P^T Diag(G_P1..G_P,n/b) Psi_P        (the same construction on the n side)
+ *   G = (I + Q)(I + Q + Q^2 + Q^3), Q = -Q^T     section 3, Cayley-Neumann
+ *   Q stored as its b(b-1)/2 upper triangle      section 3
+ * W0 (m x n) is frozen between merges; every few hundred steps the training
+ * loop folds R and P into it (W0 <- R W0 P), resets Q = 0 and draws new
+ * permutations (merge_if_needed in the write-up's API snippet).
+ *
+ * Batched row form: X is T x m (one token per row), Z = X R W0 P is T x n.
+ *
+ * Conventions shared by every call:
+ *  - Every pointer argument is a DEVICE pointer unless stated otherwise, owned
+ *    and allocated by the caller, 16-byte aligned.  The library allocates no
+ *    memory; scratch comes from the caller's workspace (`ws`, `ws_bytes`,
+ *    sized by the matching *_workspace_bytes call).
+ *  - Work is queued asynchronously on `stream` (a cudaStream_t; NULL = the
+ *    legacy default stream).  Nothing synchronises the host.
+ *  - Arguments are validated before anything is queued; on error the call
+ *    returns a non-zero poetx_status and queues nothing.  A failure reported
+ *    by the CUDA runtime while queueing returns POETX_E_CUDA.
+ *  - Kernels never trap: a wait that times out inside a kernel or an index
+ *    out of range sets a sticky device error word, read with
+ *    poetx_device_error().
+ *  - Layout of the stored weight (the "Psi frame"): W is [n][m] row-major,
+ *    W[j'][i'] = W0[permR[i']][permP[j']], i.e. the nn.Linear weight W0^T with
+ *    rows permuted by Psi_P and columns by Psi_R.  Permutations: perm[i'] is
+ *    the natural index at frame position i', (Psi v)[i'] = v[perm[i']].
+ *  - Packed triangle: row-major over i < j, k(i,j) = i(b-1) - i(i-1)/2 +
+ *    (j-i-1), Q[i][j] = +q[k], Q[j][i] = -q[k].
+ *  - dtype POETX_BF16: x, z, W, G, y_save, dz, dx are bf16, accumulation is
+ *    fp32 on tcgen05 tensor cores; b must be a multiple of 64.  dtype
+ *    POETX_FP32: everything fp32 (FFMA; tcgen05 has no fp32 kind).
+ *  - Requirements: b >= 2 divides m and n; the device is compute capability
+ *    10.0 (B200).
+ */
+#ifndef POETX_H
+#define POETX_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  POETX_OK = 0,
+  POETX_E_ARG = 1,       /* null pointer, negative size, bad flag */
+  POETX_E_SHAPE = 2,     /* b does not divide m or n, b unsupported for the dtype */
+  POETX_E_DTYPE = 3,     /* unknown dtype */
+  POETX_E_ALIGN = 4,     /* a pointer is not 16-byte aligned */
+  POETX_E_WORKSPACE = 5, /* ws too small or NULL */
+  POETX_E_ARCH = 6,      /* current device is not compute capability 10.0 */
+  POETX_E_CUDA = 7       /* the CUDA runtime reported an error while queueing */
+} poetx_status;
+
+typedef enum { POETX_FP32 = 0, POETX_BF16 = 1 } poetx_dtype;
+
+/* One layer.  All pointers are device pointers owned by the caller. */
+typedef struct {
+  int32_t m, n, b;      /* W0 is m x n; blocks of b x b */
+  int32_t dtype;        /* poetx_dtype */
+  void* W;              /* [n][m] frame-ordered frozen weight (see above) */
+  const int32_t* permR; /* [m] Psi_R */
+  const int32_t* permP; /* [n] Psi_P */
+  float* qR;            /* [m/b][b(b-1)/2] packed triangles of Q_R (fp32) */
+  float* qP;            /* [n/b][b(b-1)/2] packed triangles of Q_P (fp32) */
+  void* GR;             /* [m/b][b][b] G_R blocks in dtype, written by poetx_cnp_build */
+  void* GP;             /* [n/b][b][b] G_P blocks in dtype */
+} poetx_layer;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* poetx_status_string(int status);
+
+/* ABI version (major*10000 + minor*100 + patch). */
+int32_t poetx_version(void);
+
+/* Reads the sticky device error word (bit 1: a bounded wait inside a GEMM
+ * timed out; bit 2: a bounded wait inside a copy kernel timed out; bit 4: a
+ * permutation index was out of range) into *code (HOST pointer) and clears
+ * it.  Synchronises the current device. */
+poetx_status poetx_device_error(uint32_t* code);
+
+/* Workspace sizes in bytes (host-side arithmetic only, no device access). */
+size_t poetx_cnp_workspace_bytes(int32_t nblk, int32_t b, int32_t dtype);
+size_t poetx_forward_workspace_bytes(const poetx_layer* layer, int64_t T);
+size_t poetx_backward_workspace_bytes(const poetx_layer* layer, int64_t T);
+size_t poetx_merge_workspace_bytes(const poetx_layer* layer);
+size_t poetx_check_perm_workspace_bytes(int32_t len);
+
+/* Stored-weight frame.  import: W = frame(W0lin) with W0lin the natural
+ * nn.Linear weight W0^T ([n][m], dtype); export is the inverse.  Bit-exact
+ * permutations (section 2's Psi folded into W0's row/column order). */
+poetx_status poetx_frame_import(const poetx_layer* layer, const void* W0lin, void* stream);
+poetx_status poetx_frame_export(const poetx_layer* layer, void* W0lin, void* stream);
+
+/* Cayley-Neumann build (section 3): for each of nblk packed triangles
+ * q[nblk][b(b-1)/2] (fp32) writes G[nblk][b][b] (dtype) with
+ * G = (I+Q)(I+Q+Q^2+Q^3), evaluated as S = Q Q, G = I + 2Q + 2S + (2Q+S) S
+ * (every power of Q is built from Q and S = Q^2).  POETX_FP32: fp32 FFMA;
+ * POETX_BF16: tf32 tensor cores, fp32 accumulate, G rounded once to bf16. */
+poetx_status poetx_cnp_build(int32_t nblk, int32_t b, const float* q, int32_t dtype, void* G, void* ws,
+                             size_t ws_bytes, void* stream);
+
+/* Backward of poetx_cnp_build: given dG = dL/dG [nblk][b][b] (fp32), writes
+ * dq = dL/dq [nblk][b(b-1)/2] (fp32), dq_k = dL/dQ[i][j] - dL/dQ[j][i].
+ * accumulate != 0 adds to dq instead of overwriting it.  dtype names the
+ * layer precision the gradient serves: POETX_FP32 multiplies in fp32 FFMA,
+ * POETX_BF16 on tcgen05 tensor cores with tf32 operands (fp32 accumulate). */
+poetx_status poetx_cnp_backward(int32_t nblk, int32_t b, const float* q, const float* dG, float* dq,
+                                int32_t accumulate, int32_t dtype, void* ws, size_t ws_bytes, void* stream);
+
+/* Forward (section 1, input-centric): z = x R W0 P for T token rows.
+ * x [T][m], z [T][n] in natural feature order (dtype).  y_save [T][n] (dtype)
+ * receives Y = (x Psi_R^T Diag(G_R)) W (the P-side input, in the Psi_P
+ * frame) for the backward; pass NULL for inference.  Uses layer->GR/GP as
+ * last built by poetx_cnp_build.  T = 0 is a no-op. */
+poetx_status poetx_forward(const poetx_layer* layer, int64_t T, const void* x, void* z, void* y_save, void* ws,
+                           size_t ws_bytes, void* stream);
+
+/* Backward of L = <dz, z>: dx [T][m] (dtype; NULL skips it) and the packed
+ * gradients dqR [m/b][b(b-1)/2], dqP [n/b][b(b-1)/2] (fp32; overwritten, or
+ * added to when accumulate != 0).  Needs x and the y_save of the matching
+ * forward; W0 is frozen, so no dW0.  The dq sums over tokens use a fixed
+ * split and order (deterministic for a given shape). */
+poetx_status poetx_backward(const poetx_layer* layer, int64_t T, const void* x, const void* y_save,
+                            const void* dz, void* dx, float* dqR, float* dqP, int32_t accumulate, void* ws,
+                            size_t ws_bytes, void* stream);
+
+/* Merge (merge_if_needed in the write-up's API snippet): writes into W_out
+ * ([n][m], dtype, must not overlap layer->W) the weight R W0 P expressed in
+ * the frame of new_permR [m], new_permP [n] (device), with R and P built from
+ * the layer's current G blocks; then sets qR = qP = 0 and GR = GP = I.  The
+ * intermediate W Diag(G_R)^T is kept in fp32 (bf16 layers: the second block
+ * product reads it at tf32 precision) and rounded to dtype once at the end.
+ * The caller swaps W_out and the permutations into the layer afterwards. */
+poetx_status poetx_merge(const poetx_layer* layer, const int32_t* new_permR, const int32_t* new_permP,
+                         void* W_out, void* ws, size_t ws_bytes, void* stream);
+
+/* Debug check: *d_ok (device int32) = 1 if perm [len] is a bijection of
+ * 0..len-1, else 0. */
+poetx_status poetx_check_perm(const int32_t* perm, int32_t len, int32_t* d_ok, void* ws, size_t ws_bytes,
+                              void* stream);
+
+/* Stage profiler (tracing).  Between poetx_profile_begin() and
+ * poetx_profile_end(), every kernel the library queues is bracketed by a pair
+ * of CUDA events on its stream and tagged with its stage (permute,
+ * blockdiag_gemm, w0_gemm, dg_gemm, cnp_gemm, cnp_elementwise, dg_reduce,
+ * merge).  poetx_profile_end waits for the recorded events, writes the summed
+ * device time in ms (HOST array ms_per_stage[nstages]) and the number of
+ * launches (HOST array launches_per_stage[nstages]) per stage, and stops
+ * recording.  The events are created on first use and reused. */
+int32_t poetx_profile_stage_count(void);
+const char* poetx_profile_stage_name(int32_t stage);
+poetx_status poetx_profile_begin(void);
+poetx_status poetx_profile_end(double* ms_per_stage, int64_t* launches_per_stage, int32_t nstages);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* POETX_H */

@@ -244,28 +244,34 @@ def layer_backward(X, W0, permR, qR, permP, qP, b, dZ):
     return dX, cnp_backward(qR, b, dGR), cnp_backward(qP, b, dGP)
 
 
-def grad_G_block(X, W0, permR, GR, permP, GP, dZ, side: str, j: int):
-    """dL/dG for one block j of one side over all rows of X, computing only
-    the columns that block needs (used to check full-size runs block by
-    block).  Same chain rule as `backward`, restricted to block j."""
+def grad_G_blocks(X, W0, permR, GR, permP, GP, dZ, side: str, blocks):
+    """dL/dG for the listed blocks j of one side over all rows of X, computing
+    only the columns those blocks need (used to check full-size runs block by
+    block).  Same chain rule as `backward`, restricted to the listed blocks;
+    returns a list of b x b arrays in the order of `blocks`."""
     X = np.asarray(X, dtype=np.float64)
     dZ = np.asarray(dZ, dtype=np.float64)
     permR = np.asarray(permR, dtype=np.int64)
     permP = np.asarray(permP, dtype=np.int64)
     b = GR.shape[1]
-    A = apply_rows(X, permR, GR)
+    out = []
     if side == "P":
-        cols = permP[j * b:(j + 1) * b]
-        Yg_j = A @ W0[:, cols]
-        dV_j = dZ[:, cols]
-        return Yg_j.T @ dV_j
+        A = apply_rows(X, permR, GR)
+        for j in blocks:
+            cols = permP[j * b:(j + 1) * b]
+            Yg_j = A @ W0[:, cols]
+            dV_j = dZ[:, cols]
+            out.append(Yg_j.T @ dV_j)
+        return out
     if side != "R":
         raise ValueError("side must be 'R' or 'P'")
     dY = apply_rows_transposed(dZ, permP, GP)      # rows: dZ P^T
-    cols = permR[j * b:(j + 1) * b]
-    dU_j = dY @ W0[cols, :].T
-    Xg_j = X[:, cols]
-    return Xg_j.T @ dU_j
+    for j in blocks:
+        cols = permR[j * b:(j + 1) * b]
+        dU_j = dY @ W0[cols, :].T
+        Xg_j = X[:, cols]
+        out.append(Xg_j.T @ dU_j)
+    return out
 
 
 # --------------------------------------------------------------------------

@@ -1,0 +1,438 @@
+// Batched, split-K GEMM used by every contraction of the POET-X layer:
+//   C[t][s] = alpha * A_t(K-range s) B_t(K-range s) + beta1 X1 + beta2 X2 + diag I
+// where t runs over a batch (the b x b blocks of Diag(G_1..G_k)) and s over
+// K-splits.  Two back ends consume the same description:
+//   * tc_gemm  : tcgen05 tensor cores (kind::f16 with bf16 operands, or
+//                kind::tf32 with fp32 operands), TMA-fed, fp32 accumulators in
+//                TMEM, persistent and warp-specialised;
+//   * simt_gemm: fp32 FFMA, for the all-fp32 layer (tcgen05 has no fp32 kind).
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "ptx.cuh"
+
+namespace poetx {
+
+enum ElemType : int { ET_F32 = 0, ET_BF16 = 1 };
+
+inline int elem_size(int et) { return et == ET_BF16 ? 2 : 4; }
+
+// A 2-D row-major view of an operand (element units).  Element (mn, k) of
+// batch t sits at view coordinate
+//   K-major  (mn_major == false): row = mn + t*b_row, col = k + t*b_col
+//   MN-major (mn_major == true) : row = k + t*b_row,  col = mn + t*b_col
+// Coordinates outside [0,rows) x [0,cols) read as zero.
+struct Operand2D {
+  const void* ptr = nullptr;
+  int et = ET_BF16;
+  int64_t rows = 0, cols = 0, ld = 0;
+  bool mn_major = false;
+  int64_t b_row = 0, b_col = 0;
+};
+
+struct OutDesc {
+  void* ptr = nullptr;
+  int et = ET_BF16;
+  int64_t ld = 0;            // row stride
+  int64_t batch_stride = 0;  // element offset per batch index
+  int64_t split_stride = 0;  // element offset per K-split (partial sums)
+};
+
+struct AddDesc {
+  const float* ptr = nullptr;  // fp32, indexed like the output
+  int64_t ld = 0, batch_stride = 0;
+  float beta = 0.f;
+};
+
+struct GemmDesc {
+  int M = 0, N = 0, K = 0;
+  int batch = 1, splits = 1;
+  Operand2D A, B;
+  OutDesc C;
+  float alpha = 1.f;
+  AddDesc add1, add2;
+  float diag = 0.f;
+};
+
+// ------------------------------------------------------------------ epilogue
+struct EpiParams {
+  int M, N;
+  void* c;
+  int c_et;
+  int64_t ldc, c_bs, c_ss;
+  float alpha;
+  const float* x1;
+  int64_t x1_ld, x1_bs;
+  float beta1;
+  const float* x2;
+  int64_t x2_ld, x2_bs;
+  float beta2;
+  float diag;
+};
+
+inline EpiParams make_epi(const GemmDesc& g) {
+  EpiParams e;
+  e.M = g.M;
+  e.N = g.N;
+  e.c = g.C.ptr;
+  e.c_et = g.C.et;
+  e.ldc = g.C.ld;
+  e.c_bs = g.C.batch_stride;
+  e.c_ss = g.C.split_stride;
+  e.alpha = g.alpha;
+  e.x1 = g.add1.ptr;
+  e.x1_ld = g.add1.ld;
+  e.x1_bs = g.add1.batch_stride;
+  e.beta1 = g.add1.beta;
+  e.x2 = g.add2.ptr;
+  e.x2_ld = g.add2.ld;
+  e.x2_bs = g.add2.batch_stride;
+  e.beta2 = g.add2.beta;
+  e.diag = g.diag;
+  return e;
+}
+
+__device__ __forceinline__ float epi_value(const EpiParams& e, float acc, int t, int64_t r, int64_t n) {
+  float v = e.alpha * acc;
+  if (e.x1) v += e.beta1 * e.x1[t * e.x1_bs + r * e.x1_ld + n];
+  if (e.x2) v += e.beta2 * e.x2[t * e.x2_bs + r * e.x2_ld + n];
+  if (r == n) v += e.diag;
+  return v;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// ------------------------------------------------------------------ tcgen05 GEMM
+namespace tc {
+
+constexpr int BM = 128;
+constexpr int NUM_THREADS = 192;  // warp 0: TMA, warp 1: MMA + TMEM owner, warps 2-5: epilogue
+constexpr int GROUP_M = 16;       // M-tiles per raster group (L2 reuse of the B panel)
+
+struct Params {
+  int M, N, K, batch, splits, k_per_split;
+  int tiles_m, tiles_n;
+  int a_mn, b_mn;
+  int a_brow, a_bcol, b_brow, b_bcol;
+  uint32_t idesc;
+  uint32_t a_lbo, b_lbo, a_kstep, b_kstep;
+  EpiParams epi;
+};
+
+template <int BN, bool TF32>
+struct Cfg {
+  static constexpr int ESZ = TF32 ? 4 : 2;
+  static constexpr int CH = 128 / ESZ;  // elements per 128-byte swizzle row = K per stage
+  static constexpr int UMMA_K = TF32 ? 8 : 16;
+  static constexpr int A_BYTES = BM * 128;
+  static constexpr int B_BYTES = BN * 128;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
+  static constexpr int TMEM_COLS = 2 * BN;  // double-buffered fp32 accumulator
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+};
+
+__device__ __forceinline__ void decode_tile(const Params& p, int tile, int& bt, int& sp, int& mt, int& nt) {
+  const int per = p.tiles_m * p.tiles_n;
+  const int bs = tile / per;
+  int r = tile - bs * per;
+  bt = bs / p.splits;
+  sp = bs - bt * p.splits;
+  const int group_span = GROUP_M * p.tiles_n;
+  const int g = r / group_span;
+  const int first_m = g * GROUP_M;
+  const int gsize = min(p.tiles_m - first_m, GROUP_M);
+  r -= g * group_span;
+  mt = first_m + r % gsize;
+  nt = r / gsize;
+}
+
+template <int BN, bool TF32>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, Params p) {
+  using C = Cfg<BN, TF32>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  // bars: full[STAGES], empty[STAGES], tfull[2], tempty[2], drain
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * C::STAGES + 5);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t smem_base = smem_u32(smem);
+  auto bar = [&](int i) { return smem_u32(bars + i); };
+  const int FULL = 0, EMPTY = C::STAGES, TFULL = 2 * C::STAGES, TEMPTY = 2 * C::STAGES + 2,
+            DRAIN = 2 * C::STAGES + 4;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(bar(FULL + s), 1);
+      mbar_init(bar(EMPTY + s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(bar(TFULL + a), 1);
+      mbar_init(bar(TEMPTY + a), 128);
+    }
+    mbar_init(bar(DRAIN), 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  const int total = p.batch * p.splits * p.tiles_m * p.tiles_n;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer
+      prefetch_tmap(&tmA);
+      prefetch_tmap(&tmB);
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed = 0, armed_phase = 0;  // per-stage bits for the abort drain
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        int bt, sp, mt, nt;
+        decode_tile(p, tile, bt, sp, mt, nt);
+        const int kbeg = sp * p.k_per_split;
+        const int kend = min(p.K, kbeg + p.k_per_split);
+        const int nkb = (kend - kbeg + C::CH - 1) / C::CH;
+        const int m0 = mt * BM, n0 = nt * BN;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(bar(EMPTY + stage), phase ^ 1u, DERR_GEMM_WAIT)) { ok = false; break; }
+          const uint32_t fb = bar(FULL + stage);
+          mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
+          armed |= 1u << stage;
+          armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
+          const uint32_t sa = smem_base + stage * C::STAGE_BYTES;
+          const uint32_t sb = sa + C::A_BYTES;
+          const int k = kbeg + kb * C::CH;
+          if (!p.a_mn) {
+            tma_load_2d(sa, &tmA, fb, k + bt * p.a_bcol, m0 + bt * p.a_brow);
+          } else {
+#pragma unroll
+            for (int c = 0; c < BM / C::CH; ++c)
+              tma_load_2d(sa + c * (C::CH * 128), &tmA, fb, m0 + c * C::CH + bt * p.a_bcol, k + bt * p.a_brow);
+          }
+          if (!p.b_mn) {
+            tma_load_2d(sb, &tmB, fb, k + bt * p.b_bcol, n0 + bt * p.b_brow);
+          } else {
+#pragma unroll
+            for (int c = 0; c < BN / C::CH; ++c)
+              tma_load_2d(sb + c * (C::CH * 128), &tmB, fb, n0 + c * C::CH + bt * p.b_bcol, k + bt * p.b_brow);
+          }
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        // Let the copies already issued land before the block exits.
+        for (int s = 0; s < C::STAGES; ++s)
+          if (armed & (1u << s)) mbar_wait(bar(FULL + s), (armed_phase >> s) & 1u, DERR_GEMM_WAIT);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer
+      const uint32_t a_base_lbo = p.a_lbo, b_base_lbo = p.b_lbo;
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++local) {
+        int bt, sp, mt, nt;
+        decode_tile(p, tile, bt, sp, mt, nt);
+        const int kbeg = sp * p.k_per_split;
+        const int kend = min(p.K, kbeg + p.k_per_split);
+        const int nkb = (kend - kbeg + C::CH - 1) / C::CH;
+        const int acc = local & 1;
+        const uint32_t acc_phase = (local >> 1) & 1;
+        if (!mbar_wait(bar(TEMPTY + acc), acc_phase ^ 1u, DERR_GEMM_WAIT)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(bar(FULL + stage), phase, DERR_GEMM_WAIT)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_base + stage * C::STAGE_BYTES;
+          const uint32_t sb = sa + C::A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < C::CH / C::UMMA_K; ++kk) {
+            const uint64_t da = smem_desc_sw128(sa + kk * p.a_kstep, a_base_lbo, 1024);
+            const uint64_t db = smem_desc_sw128(sb + kk * p.b_kstep, b_base_lbo, 1024);
+            tc_mma<TF32>(d_tmem, da, db, p.idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          tc_commit(bar(EMPTY + stage));
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit(bar(TFULL + acc));
+      }
+      // All MMAs issued by this thread have completed once DRAIN fires.
+      tc_commit(bar(DRAIN));
+      mbar_wait(bar(DRAIN), 0, DERR_GEMM_WAIT);
+    }
+  } else {
+    // ---------------- epilogue: TMEM -> registers -> global
+    const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter + 32)
+    const EpiParams& e = p.epi;
+    int local = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
+      int bt, sp, mt, nt;
+      decode_tile(p, tile, bt, sp, mt, nt);
+      const int acc = local & 1;
+      const uint32_t acc_phase = (local >> 1) & 1;
+      bool ok = mbar_wait(bar(TFULL + acc), acc_phase, DERR_GEMM_WAIT);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const int64_t r = static_cast<int64_t>(mt) * BM + quarter * 32 + lane;
+      const bool row_ok = r < e.M;
+      const int64_t obase = bt * e.c_bs + sp * e.c_ss + r * e.ldc;
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        float v[32];
+        tmem_ld_32cols(tmem_base + acc * BN + c0 + (static_cast<uint32_t>(quarter * 32) << 16), v);
+        const int64_t n0 = static_cast<int64_t>(nt) * BN + c0;
+        if (!row_ok) continue;
+        if (n0 + 32 <= e.N) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = epi_value(e, v[i], bt, r, n0 + i);
+          if (e.c_et == ET_BF16) {
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(e.c) + obase + n0);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              dst[q] = make_uint4(pack_bf16x2(v[8 * q + 0], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                                  pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+          } else {
+            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(e.c) + obase + n0);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+          }
+        } else {
+          for (int i = 0; i < 32 && n0 + i < e.N; ++i) {
+            const float o = epi_value(e, v[i], bt, r, n0 + i);
+            if (e.c_et == ET_BF16)
+              reinterpret_cast<__nv_bfloat16*>(e.c)[obase + n0 + i] = __float2bfloat16_rn(o);
+            else
+              reinterpret_cast<float*>(e.c)[obase + n0 + i] = o;
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(TEMPTY + acc));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+}  // namespace tc
+
+// ------------------------------------------------------------------ SIMT fp32 GEMM
+namespace simt {
+
+constexpr int TM = 64, TN = 64, TK = 16, THREADS = 256;
+
+struct Params {
+  int M, N, K, splits, k_per_split;
+  const float* a;
+  int64_t a_rows, a_cols, a_ld, a_brow, a_bcol;
+  int a_mn;
+  const float* b;
+  int64_t b_rows, b_cols, b_ld, b_brow, b_bcol;
+  int b_mn;
+  EpiParams epi;
+};
+
+__device__ __forceinline__ float load_op(const float* base, int64_t rows, int64_t cols, int64_t ld, int64_t brow,
+                                         int64_t bcol, int mn_major, int t, int64_t mn, int64_t k) {
+  int64_t row, col;
+  if (mn_major) {
+    row = k + t * brow;
+    col = mn + t * bcol;
+  } else {
+    row = mn + t * brow;
+    col = k + t * bcol;
+  }
+  if (row < 0 || row >= rows || col < 0 || col >= cols) return 0.f;
+  return base[row * ld + col];
+}
+
+__global__ void __launch_bounds__(THREADS) gemm_kernel(Params p) {
+  __shared__ float As[TK][TM + 4];
+  __shared__ float Bs[TK][TN + 4];
+  const int bz = blockIdx.z;
+  const int t = bz / p.splits;
+  const int sp = bz - t * p.splits;
+  const int m0 = blockIdx.y * TM, n0 = blockIdx.x * TN;
+  const int kbeg = sp * p.k_per_split;
+  const int kend = min(p.K, kbeg + p.k_per_split);
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+  float acc[4][4] = {};
+  for (int k0 = kbeg; k0 < kend; k0 += TK) {
+    for (int i = threadIdx.x; i < TK * TM; i += THREADS) {
+      const int kk = i / TM, mm = i % TM;
+      const int64_t mg = m0 + mm, kg = k0 + kk;
+      As[kk][mm] = (mg < p.M && kg < kend)
+                       ? load_op(p.a, p.a_rows, p.a_cols, p.a_ld, p.a_brow, p.a_bcol, p.a_mn, t, mg, kg)
+                       : 0.f;
+    }
+    for (int i = threadIdx.x; i < TK * TN; i += THREADS) {
+      const int kk = i / TN, nn = i % TN;
+      const int64_t ng = n0 + nn, kg = k0 + kk;
+      Bs[kk][nn] = (ng < p.N && kg < kend)
+                       ? load_op(p.b, p.b_rows, p.b_cols, p.b_ld, p.b_brow, p.b_bcol, p.b_mn, t, ng, kg)
+                       : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < TK; ++kk) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = As[kk][ty * 4 + i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) b[j] = Bs[kk][tx * 4 + j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+  const EpiParams& e = p.epi;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t r = m0 + ty * 4 + i;
+    if (r >= e.M) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int64_t n = n0 + tx * 4 + j;
+      if (n >= e.N) continue;
+      const float v = epi_value(e, acc[i][j], t, r, n);
+      const int64_t o = t * e.c_bs + sp * e.c_ss + r * e.ldc + n;
+      if (e.c_et == ET_BF16)
+        reinterpret_cast<__nv_bfloat16*>(e.c)[o] = __float2bfloat16_rn(v);
+      else
+        reinterpret_cast<float*>(e.c)[o] = v;
+    }
+  }
+}
+
+}  // namespace simt
+}  // namespace poetx

@@ -1,0 +1,166 @@
+// Host side of the batched GEMM: tensor-map encoding, tile-shape choice,
+// split-K sizing and launch of the tcgen05 or SIMT back end.
+#pragma once
+
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "gemm.cuh"
+
+namespace poetx {
+
+// cuTensorMapEncodeTiled from the driver, fetched through the runtime so the
+// library links against cudart only.
+inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+inline int sm_count(int device) {
+  static int counts[64] = {0};
+  if (device < 0 || device >= 64) return 148;
+  if (counts[device] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || v <= 0) v = 148;
+    counts[device] = v;
+  }
+  return counts[device];
+}
+
+// 2-D tensor map over a row-major view with a 128-byte swizzled box of
+// (box_inner elements = 128 bytes) x box_outer rows.
+inline bool encode_map(CUtensorMap* map, const Operand2D& op, int box_outer) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  const int esz = elem_size(op.et);
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(op.cols), static_cast<cuuint64_t>(op.rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(op.ld) * esz};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esz), static_cast<cuuint32_t>(box_outer)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, op.et == ET_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+                   const_cast<void*>(op.ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Split-K count so that (tiles x splits) fills about `waves` of the SMs while
+// every split keeps at least `min_kb` K-blocks.
+inline int choose_splits(int tiles, int K, int kblock, int sms, int min_kb = 4) {
+  const int nkb = (K + kblock - 1) / kblock;
+  int s = 1;
+  while (tiles * s * 2 <= sms * 2 && nkb / (s * 2) >= min_kb) s *= 2;
+  while (tiles * s < sms && nkb / (s + 1) >= min_kb) ++s;
+  return s;
+}
+
+template <int BN, bool TF32>
+cudaError_t launch_tc_typed(const GemmDesc& g, cudaStream_t st, int device) {
+  using C = tc::Cfg<BN, TF32>;
+  static bool attr_set[64] = {false};
+  if (device >= 0 && device < 64 && !attr_set[device]) {
+    cudaError_t e =
+        cudaFuncSetAttribute(tc::gemm_kernel<BN, TF32>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set[device] = true;
+  }
+  CUtensorMap ma, mb;
+  if (!encode_map(&ma, g.A, g.A.mn_major ? C::CH : tc::BM)) return cudaErrorInvalidValue;
+  if (!encode_map(&mb, g.B, g.B.mn_major ? C::CH : BN)) return cudaErrorInvalidValue;
+  tc::Params p;
+  p.M = g.M;
+  p.N = g.N;
+  p.K = g.K;
+  p.batch = g.batch;
+  p.splits = g.splits;
+  const int nkb = (g.K + C::CH - 1) / C::CH;
+  const int kb_per = (nkb + g.splits - 1) / g.splits;
+  p.k_per_split = kb_per * C::CH;
+  p.tiles_m = (g.M + tc::BM - 1) / tc::BM;
+  p.tiles_n = (g.N + BN - 1) / BN;
+  p.a_mn = g.A.mn_major;
+  p.b_mn = g.B.mn_major;
+  p.a_brow = static_cast<int>(g.A.b_row);
+  p.a_bcol = static_cast<int>(g.A.b_col);
+  p.b_brow = static_cast<int>(g.B.b_row);
+  p.b_bcol = static_cast<int>(g.B.b_col);
+  const uint32_t fmt = TF32 ? 2u : 1u;
+  p.idesc = (1u << 4) | (fmt << 7) | (fmt << 10) | (static_cast<uint32_t>(g.A.mn_major) << 15) |
+            (static_cast<uint32_t>(g.B.mn_major) << 16) | (static_cast<uint32_t>(BN >> 3) << 17) |
+            (static_cast<uint32_t>(tc::BM >> 4) << 24);
+  // K-major: the K step of one MMA is 32 bytes inside the 128-byte row; the
+  // leading offset is unused.  MN-major: one MMA spans UMMA_K rows of 128
+  // bytes; 128-byte MN chunks sit one box (CH rows x 128 B) apart.
+  p.a_kstep = g.A.mn_major ? C::UMMA_K * 128 : 32;
+  p.b_kstep = g.B.mn_major ? C::UMMA_K * 128 : 32;
+  p.a_lbo = g.A.mn_major ? C::CH * 128 : 16;
+  p.b_lbo = g.B.mn_major ? C::CH * 128 : 16;
+  p.epi = make_epi(g);
+  const int total = g.batch * g.splits * p.tiles_m * p.tiles_n;
+  const int grid = total < sm_count(device) ? total : sm_count(device);
+  if (grid <= 0) return cudaSuccess;
+  tc::gemm_kernel<BN, TF32><<<grid, tc::NUM_THREADS, C::SMEM_BYTES, st>>>(ma, mb, p);
+  return cudaGetLastError();
+}
+
+// The N tile: the widest of 256/128/64 that divides N (N is a multiple of 64
+// on the tensor-core path).
+inline int choose_bn(int N) {
+  if (N % 256 == 0) return 256;
+  if (N % 128 == 0) return 128;
+  return 64;
+}
+
+inline cudaError_t launch_tc(const GemmDesc& g, cudaStream_t st, int device) {
+  const bool tf32 = g.A.et == ET_F32;
+  switch (choose_bn(g.N)) {
+    case 256: return tf32 ? launch_tc_typed<256, true>(g, st, device) : launch_tc_typed<256, false>(g, st, device);
+    case 128: return tf32 ? launch_tc_typed<128, true>(g, st, device) : launch_tc_typed<128, false>(g, st, device);
+    default: return tf32 ? launch_tc_typed<64, true>(g, st, device) : launch_tc_typed<64, false>(g, st, device);
+  }
+}
+
+inline cudaError_t launch_simt(const GemmDesc& g, cudaStream_t st) {
+  simt::Params p;
+  p.M = g.M;
+  p.N = g.N;
+  p.K = g.K;
+  p.splits = g.splits;
+  const int nkb = (g.K + simt::TK - 1) / simt::TK;
+  p.k_per_split = ((nkb + g.splits - 1) / g.splits) * simt::TK;
+  p.a = static_cast<const float*>(g.A.ptr);
+  p.a_rows = g.A.rows;
+  p.a_cols = g.A.cols;
+  p.a_ld = g.A.ld;
+  p.a_brow = g.A.b_row;
+  p.a_bcol = g.A.b_col;
+  p.a_mn = g.A.mn_major;
+  p.b = static_cast<const float*>(g.B.ptr);
+  p.b_rows = g.B.rows;
+  p.b_cols = g.B.cols;
+  p.b_ld = g.B.ld;
+  p.b_brow = g.B.b_row;
+  p.b_bcol = g.B.b_col;
+  p.b_mn = g.B.mn_major;
+  p.epi = make_epi(g);
+  dim3 grid((g.N + simt::TN - 1) / simt::TN, (g.M + simt::TM - 1) / simt::TM, g.batch * g.splits);
+  if (grid.x == 0 || grid.y == 0 || grid.z == 0) return cudaSuccess;
+  simt::gemm_kernel<<<grid, simt::THREADS, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+// Tensor cores for bf16 and tf32 operands, FFMA for an all-fp32 layer.
+inline cudaError_t launch_gemm(const GemmDesc& g, bool tensor_cores, cudaStream_t st, int device) {
+  return tensor_cores ? launch_tc(g, st, device) : launch_simt(g, st);
+}
+
+}  // namespace poetx

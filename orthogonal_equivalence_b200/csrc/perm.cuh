@@ -1,0 +1,219 @@
+// Permutation traffic of the layer (POET-X write-up, section 2: R = Psi^T
+// Diag(G) Psi).  With perm[i'] the natural index at Psi-frame position i':
+//   gather : out[r][c]            = in[rowmap? rowmap[r] : r][colmap[c]]
+//   scatter: out[rowmap? rowmap[r] : r][colmap[c]] = in[r][c]
+// A block stages whole rows in shared memory, so global reads and writes are
+// contiguous 16-byte vectors and only the shared-memory side is permuted.
+// Out-of-range indices are skipped (zero written) and flagged in the device
+// error word.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+
+namespace poetx {
+
+template <typename T>
+__device__ __forceinline__ float to_f32(T v);
+template <>
+__device__ __forceinline__ float to_f32<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+template <typename T>
+__device__ __forceinline__ T from_f32(float v);
+template <>
+__device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+
+template <typename Tin, typename Tout>
+__device__ __forceinline__ Tout convert(Tin v) {
+  if constexpr (std::is_same<Tin, Tout>::value) return v;
+  else return from_f32<Tout>(to_f32<Tin>(v));
+}
+
+// Copy `count` elements of a row into shared memory (16-byte vectors when the
+// row is 16-byte aligned and a whole number of vectors).
+template <typename T>
+__device__ __forceinline__ void row_to_smem(const T* __restrict__ src, T* dst, int count) {
+  constexpr int V = 16 / sizeof(T);
+  if ((reinterpret_cast<uintptr_t>(src) & 15u) == 0 && count % V == 0) {
+    const uint4* s4 = reinterpret_cast<const uint4*>(src);
+    uint4* d4 = reinterpret_cast<uint4*>(dst);
+    for (int i = threadIdx.x; i < count / V; i += blockDim.x) d4[i] = __ldg(s4 + i);
+  } else {
+    for (int i = threadIdx.x; i < count; i += blockDim.x) dst[i] = src[i];
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ void smem_to_row(const T* src, T* __restrict__ dst, int count) {
+  constexpr int V = 16 / sizeof(T);
+  if ((reinterpret_cast<uintptr_t>(dst) & 15u) == 0 && count % V == 0) {
+    const uint4* s4 = reinterpret_cast<const uint4*>(src);
+    uint4* d4 = reinterpret_cast<uint4*>(dst);
+    for (int i = threadIdx.x; i < count / V; i += blockDim.x) d4[i] = s4[i];
+  } else {
+    for (int i = threadIdx.x; i < count; i += blockDim.x) dst[i] = src[i];
+  }
+}
+
+// rows_per_iter rows are staged per pass (shared memory = rows_per_iter *
+// cols * sizeof(Tin)).
+template <typename Tin, typename Tout>
+__global__ void __launch_bounds__(256) gather_kernel(const Tin* __restrict__ in, int64_t ld_in, int64_t in_rows,
+                                                     Tout* __restrict__ out, int64_t ld_out, int64_t rows, int cols,
+                                                     const int32_t* __restrict__ colmap,
+                                                     const int32_t* __restrict__ rowmap, int rows_per_iter) {
+  extern __shared__ __align__(16) uint8_t sm_raw[];
+  Tin* sm = reinterpret_cast<Tin*>(sm_raw);
+  constexpr int VO = 16 / sizeof(Tout);
+  const bool vec_out = (cols % VO == 0) && (ld_out % VO == 0) && ((reinterpret_cast<uintptr_t>(out) & 15u) == 0);
+  for (int64_t r0 = static_cast<int64_t>(blockIdx.x) * rows_per_iter; r0 < rows;
+       r0 += static_cast<int64_t>(gridDim.x) * rows_per_iter) {
+    const int nr = static_cast<int>(rows - r0 < rows_per_iter ? rows - r0 : rows_per_iter);
+    for (int q = 0; q < nr; ++q) {
+      int64_t sr = r0 + q;
+      if (rowmap) sr = rowmap[sr];
+      if (sr < 0 || sr >= in_rows) {
+        if (threadIdx.x == 0) record_error(DERR_BAD_INDEX);
+        for (int i = threadIdx.x; i < cols; i += blockDim.x) sm[q * cols + i] = Tin(0.f);
+      } else {
+        row_to_smem(in + sr * ld_in, sm + q * cols, cols);
+      }
+    }
+    __syncthreads();
+    for (int q = 0; q < nr; ++q) {
+      const Tin* srow = sm + q * cols;
+      Tout* orow = out + (r0 + q) * ld_out;
+      if (vec_out) {
+        for (int v = threadIdx.x; v < cols / VO; v += blockDim.x) {
+          union {
+            uint4 u;
+            Tout e[VO];
+          } pk;
+#pragma unroll
+          for (int i = 0; i < VO; ++i) {
+            const int s = colmap[v * VO + i];
+            if (s < 0 || s >= cols) {
+              record_error(DERR_BAD_INDEX);
+              pk.e[i] = from_f32<Tout>(0.f);
+            } else {
+              pk.e[i] = convert<Tin, Tout>(srow[s]);
+            }
+          }
+          reinterpret_cast<uint4*>(orow)[v] = pk.u;
+        }
+      } else {
+        for (int c = threadIdx.x; c < cols; c += blockDim.x) {
+          const int s = colmap[c];
+          if (s < 0 || s >= cols) {
+            record_error(DERR_BAD_INDEX);
+            orow[c] = from_f32<Tout>(0.f);
+          } else {
+            orow[c] = convert<Tin, Tout>(srow[s]);
+          }
+        }
+      }
+    }
+    __syncthreads();
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) scatter_kernel(const T* __restrict__ in, int64_t ld_in, T* __restrict__ out,
+                                                      int64_t ld_out, int64_t out_rows, int64_t rows, int cols,
+                                                      const int32_t* __restrict__ colmap,
+                                                      const int32_t* __restrict__ rowmap, int rows_per_iter) {
+  extern __shared__ __align__(16) uint8_t sm_raw[];
+  T* sm = reinterpret_cast<T*>(sm_raw);
+  constexpr int V = 16 / sizeof(T);
+  const bool vec_in = (cols % V == 0) && (ld_in % V == 0) && ((reinterpret_cast<uintptr_t>(in) & 15u) == 0);
+  for (int64_t r0 = static_cast<int64_t>(blockIdx.x) * rows_per_iter; r0 < rows;
+       r0 += static_cast<int64_t>(gridDim.x) * rows_per_iter) {
+    const int nr = static_cast<int>(rows - r0 < rows_per_iter ? rows - r0 : rows_per_iter);
+    for (int q = 0; q < nr; ++q) {
+      const T* irow = in + (r0 + q) * ld_in;
+      T* srow = sm + q * cols;
+      if (vec_in) {
+        for (int v = threadIdx.x; v < cols / V; v += blockDim.x) {
+          union {
+            uint4 u;
+            T e[V];
+          } pk;
+          pk.u = __ldg(reinterpret_cast<const uint4*>(irow) + v);
+#pragma unroll
+          for (int i = 0; i < V; ++i) {
+            const int d = colmap[v * V + i];
+            if (d < 0 || d >= cols) record_error(DERR_BAD_INDEX);
+            else srow[d] = pk.e[i];
+          }
+        }
+      } else {
+        for (int c = threadIdx.x; c < cols; c += blockDim.x) {
+          const int d = colmap[c];
+          if (d < 0 || d >= cols) record_error(DERR_BAD_INDEX);
+          else srow[d] = irow[c];
+        }
+      }
+    }
+    __syncthreads();
+    for (int q = 0; q < nr; ++q) {
+      int64_t dr = r0 + q;
+      if (rowmap) dr = rowmap[dr];
+      if (dr < 0 || dr >= out_rows) {
+        if (threadIdx.x == 0) record_error(DERR_BAD_INDEX);
+        continue;
+      }
+      smem_to_row(sm + q * cols, out + dr * ld_out, cols);
+    }
+    __syncthreads();
+  }
+}
+
+// inv[perm[i]] = i
+__global__ void invert_perm_kernel(const int32_t* __restrict__ perm, int32_t* __restrict__ inv, int len) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= len) return;
+  const int p = perm[i];
+  if (p < 0 || p >= len) {
+    record_error(DERR_BAD_INDEX);
+    return;
+  }
+  inv[p] = i;
+}
+
+// out[i] = a[b[i]]
+__global__ void compose_perm_kernel(const int32_t* __restrict__ a, const int32_t* __restrict__ b,
+                                    int32_t* __restrict__ out, int len) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= len) return;
+  const int j = b[i];
+  if (j < 0 || j >= len) {
+    record_error(DERR_BAD_INDEX);
+    out[i] = 0;
+    return;
+  }
+  out[i] = a[j];
+}
+
+__global__ void perm_histogram_kernel(const int32_t* __restrict__ perm, int32_t* hist, int len, int32_t* ok) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= len) return;
+  const int p = perm[i];
+  if (p < 0 || p >= len) {
+    *ok = 0;
+    return;
+  }
+  atomicAdd(hist + p, 1);
+}
+
+__global__ void perm_check_kernel(const int32_t* __restrict__ hist, int len, int32_t* ok) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < len && hist[i] != 1) *ok = 0;
+}
+
+}  // namespace poetx

@@ -1,0 +1,918 @@
+// C ABI of the POET-X layer (declared in include/poetx.h): argument
+// validation, workspace carving and the launch sequence of each call on the
+// caller's stream.  The arithmetic lives in the kernels of gemm.cuh, perm.cuh
+// and cnp.cuh.
+//
+// Source of the method: POET-X write-up (zhichai.net), sections 1 (input-
+// centric layer), 2 (block-stochastic R, P), 3 (Cayley-Neumann blocks,
+// packed triangle) and the merge_if_needed step of its API snippet.
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <utility>
+#include <vector>
+
+#include "poetx.h"
+#include "cnp.cuh"
+#include "gemm_host.cuh"
+#include "perm.cuh"
+
+using namespace poetx;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr int kSplitSMs = 148;  // fixed split-K target (B200 SM count): sums do not depend on the device
+
+inline size_t al(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline int dtype_size(int32_t dt) { return dt == POETX_BF16 ? 2 : 4; }
+inline int elem_type(int32_t dt) { return dt == POETX_BF16 ? ET_BF16 : ET_F32; }
+
+struct Carver {
+  uint8_t* base;
+  size_t cap, used = 0;
+  Carver(void* b, size_t c) : base(static_cast<uint8_t*>(b)), cap(c) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(base);
+    const uintptr_t r = (a + kAlign - 1) & ~uintptr_t(kAlign - 1);
+    used = r - a;
+  }
+  template <typename T>
+  T* take(size_t bytes) {
+    T* p = reinterpret_cast<T*>(base + used);
+    used += al(bytes);
+    return p;
+  }
+};
+
+#define POETX_TRY(expr)                         \
+  do {                                          \
+    const poetx_status _s = (expr);             \
+    if (_s != POETX_OK) return _s;              \
+  } while (0)
+#define POETX_CUDA(expr)                        \
+  do {                                          \
+    if ((expr) != cudaSuccess) {                \
+      (void)cudaGetLastError();                 \
+      return POETX_E_CUDA;                      \
+    }                                           \
+  } while (0)
+
+poetx_status current_device(int* dev) {
+  if (cudaGetDevice(dev) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return POETX_E_CUDA;
+  }
+  static int cc[64] = {0};
+  if (*dev < 0 || *dev >= 64) return POETX_E_ARCH;
+  if (cc[*dev] == 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, *dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, *dev) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return POETX_E_CUDA;
+    }
+    cc[*dev] = major * 10 + minor;
+  }
+  return cc[*dev] == 100 ? POETX_OK : POETX_E_ARCH;
+}
+
+poetx_status check_dtype_b(int32_t dtype, int32_t b) {
+  if (dtype != POETX_FP32 && dtype != POETX_BF16) return POETX_E_DTYPE;
+  if (b < 2) return POETX_E_SHAPE;
+  if (dtype == POETX_BF16 && b % 64 != 0) return POETX_E_SHAPE;
+  return POETX_OK;
+}
+
+poetx_status check_layer(const poetx_layer* L) {
+  if (!L) return POETX_E_ARG;
+  POETX_TRY(check_dtype_b(L->dtype, L->b));
+  if (L->m <= 0 || L->n <= 0 || L->m % L->b != 0 || L->n % L->b != 0) return POETX_E_SHAPE;
+  const void* ptrs[] = {L->W, L->permR, L->permP, L->qR, L->qP, L->GR, L->GP};
+  for (const void* p : ptrs) {
+    if (!p) return POETX_E_ARG;
+    if (!aligned16(p)) return POETX_E_ALIGN;
+  }
+  return POETX_OK;
+}
+
+poetx_status check_ptr(const void* p) {
+  if (!p) return POETX_E_ARG;
+  return aligned16(p) ? POETX_OK : POETX_E_ALIGN;
+}
+
+
+// ---------------------------------------------------------------- stage profiler
+// When enabled (poetx_profile_begin), every kernel launch is bracketed by a
+// pair of CUDA events on its stream, tagged with the stage it belongs to;
+// poetx_profile_end sums the elapsed times per stage.
+enum Stage : int {
+  ST_PERMUTE = 0,
+  ST_BLOCKDIAG,
+  ST_W0,
+  ST_DG,
+  ST_CNP_GEMM,
+  ST_CNP_ELEM,
+  ST_REDUCE,
+  ST_MERGE,
+  ST_COUNT
+};
+const char* const kStageNames[ST_COUNT] = {"permute",  "blockdiag_gemm",  "w0_gemm",   "dg_gemm",
+                                           "cnp_gemm", "cnp_elementwise", "dg_reduce", "merge"};
+
+struct Profiler {
+  std::mutex mu;
+  bool on = false;
+  std::vector<cudaEvent_t> pool;
+  size_t used = 0;
+  std::vector<std::pair<int, size_t>> recs;  // (stage, index of the start event)
+};
+
+Profiler& profiler() {
+  static Profiler p;
+  return p;
+}
+
+struct Prof {
+  int stage;
+  cudaStream_t st;
+  size_t idx = SIZE_MAX;
+  Prof(int s, cudaStream_t stream) : stage(s), st(stream) {
+    Profiler& P = profiler();
+    std::lock_guard<std::mutex> g(P.mu);
+    if (!P.on) return;
+    while (P.used + 2 > P.pool.size()) {
+      cudaEvent_t e;
+      if (cudaEventCreate(&e) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return;
+      }
+      P.pool.push_back(e);
+    }
+    idx = P.used;
+    P.used += 2;
+    cudaEventRecord(P.pool[idx], st);
+  }
+  ~Prof() {
+    if (idx == SIZE_MAX) return;
+    Profiler& P = profiler();
+    std::lock_guard<std::mutex> g(P.mu);
+    cudaEventRecord(P.pool[idx + 1], st);
+    P.recs.emplace_back(stage, idx);
+  }
+};
+
+#define PROFILED(stage, st, ...)  \
+  do {                            \
+    Prof _prof((stage), (st));    \
+    __VA_ARGS__;                  \
+  } while (0)
+
+// ---------------------------------------------------------------- sizing
+inline bool use_tc(int32_t dtype) { return dtype == POETX_BF16; }
+
+// K-splits of the dG = Y_j^T dV_j contractions (K = T tokens): enough
+// (blocks x tiles x splits) to fill one wave, at least 4 K-blocks per split.
+int dg_splits(int nblk, int b, int64_t T, int32_t dtype) {
+  int tiles, kblock;
+  if (use_tc(dtype)) {
+    tiles = nblk * ((b + tc::BM - 1) / tc::BM) * ((b + choose_bn(b) - 1) / choose_bn(b));
+    kblock = 64;
+  } else {
+    tiles = nblk * ((b + simt::TM - 1) / simt::TM) * ((b + simt::TN - 1) / simt::TN);
+    kblock = simt::TK;
+  }
+  const int64_t nkb = (T + kblock - 1) / kblock;
+  int64_t s = kSplitSMs / (tiles > 0 ? tiles : 1);
+  if (s > nkb / 4) s = nkb / 4;
+  if (s > 32) s = 32;
+  if (s < 1) s = 1;
+  return static_cast<int>(s);
+}
+
+size_t cnp_build_ws(int32_t nblk, int32_t b) { return 3 * al(sizeof(float) * size_t(nblk) * b * b); }
+size_t cnp_bwd_ws(int32_t nblk, int32_t b) { return 7 * al(sizeof(float) * size_t(nblk) * b * b); }
+
+size_t fwd_ws(const poetx_layer* L, int64_t T) {
+  const size_t es = dtype_size(L->dtype);
+  return kAlign + 2 * al(es * T * L->m) + 2 * al(es * T * L->n);
+}
+
+size_t bwd_ws(const poetx_layer* L, int64_t T) {
+  const size_t es = dtype_size(L->dtype);
+  const int64_t mx = L->m > L->n ? L->m : L->n;
+  const int nR = L->m / L->b, nP = L->n / L->b;
+  const int nmax = nR > nP ? nR : nP;
+  const size_t bb = size_t(L->b) * L->b;
+  return kAlign + 2 * al(es * T * mx) + al(es * T * L->m) +
+         al(sizeof(float) * dg_splits(nP, L->b, T, L->dtype) * nP * bb) +
+         al(sizeof(float) * dg_splits(nR, L->b, T, L->dtype) * nR * bb) + al(sizeof(float) * nmax * bb) +
+         cnp_bwd_ws(nmax, L->b);
+}
+
+size_t merge_ws(const poetx_layer* L) {
+  const size_t nm = size_t(L->n) * L->m;
+  const int nP = L->n / L->b;
+  return kAlign + 2 * al(sizeof(float) * nm) + al(sizeof(float) * size_t(nP) * L->b * L->b) +
+         2 * al(sizeof(int32_t) * L->m) + 2 * al(sizeof(int32_t) * L->n);
+}
+
+// ---------------------------------------------------------------- launch helpers
+int grid_for(int64_t n, int threads, int device) {
+  int64_t g = (n + threads - 1) / threads;
+  const int64_t cap = int64_t(sm_count(device)) * 16;
+  if (g > cap) g = cap;
+  return g < 1 ? 1 : static_cast<int>(g);
+}
+
+template <typename K>
+cudaError_t allow_smem(K kernel, size_t bytes, bool* done) {
+  if (bytes <= 48 * 1024 || *done) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+  if (e == cudaSuccess) *done = true;
+  return e;
+}
+
+int rows_per_iter(int cols, size_t esz) {
+  const size_t row = cols * esz;
+  int r = static_cast<int>((40 * 1024) / (row ? row : 1));
+  if (r > 8) r = 8;
+  return r < 1 ? 1 : r;
+}
+
+template <typename Tin, typename Tout>
+cudaError_t gather(const Tin* in, int64_t ld_in, int64_t in_rows, Tout* out, int64_t ld_out, int64_t rows, int cols,
+                   const int32_t* colmap, const int32_t* rowmap, cudaStream_t st, int device) {
+  if (rows <= 0 || cols <= 0) return cudaSuccess;
+  static bool attr[64] = {false};
+  const int rpi = rows_per_iter(cols, sizeof(Tin));
+  const size_t smem = size_t(rpi) * cols * sizeof(Tin);
+  if (smem > 200 * 1024) return cudaErrorInvalidValue;
+  cudaError_t e = allow_smem(gather_kernel<Tin, Tout>, smem, &attr[device & 63]);
+  if (e != cudaSuccess) return e;
+  int64_t g = (rows + rpi - 1) / rpi;
+  const int64_t cap = int64_t(sm_count(device)) * 8;
+  if (g > cap) g = cap;
+  gather_kernel<Tin, Tout><<<static_cast<int>(g), 256, smem, st>>>(in, ld_in, in_rows, out, ld_out, rows, cols,
+                                                                    colmap, rowmap, rpi);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t scatter(const T* in, int64_t ld_in, T* out, int64_t ld_out, int64_t out_rows, int64_t rows, int cols,
+                    const int32_t* colmap, const int32_t* rowmap, cudaStream_t st, int device) {
+  if (rows <= 0 || cols <= 0) return cudaSuccess;
+  static bool attr[64] = {false};
+  const int rpi = rows_per_iter(cols, sizeof(T));
+  const size_t smem = size_t(rpi) * cols * sizeof(T);
+  if (smem > 200 * 1024) return cudaErrorInvalidValue;
+  cudaError_t e = allow_smem(scatter_kernel<T>, smem, &attr[device & 63]);
+  if (e != cudaSuccess) return e;
+  int64_t g = (rows + rpi - 1) / rpi;
+  const int64_t cap = int64_t(sm_count(device)) * 8;
+  if (g > cap) g = cap;
+  scatter_kernel<T><<<static_cast<int>(g), 256, smem, st>>>(in, ld_in, out, ld_out, out_rows, rows, cols, colmap,
+                                                             rowmap, rpi);
+  return cudaGetLastError();
+}
+
+cudaError_t gather_dt(int32_t dt, const void* in, int64_t ld_in, int64_t in_rows, void* out, int64_t ld_out,
+                      int64_t rows, int cols, const int32_t* colmap, const int32_t* rowmap, cudaStream_t st,
+                      int device) {
+  if (dt == POETX_BF16)
+    return gather(static_cast<const __nv_bfloat16*>(in), ld_in, in_rows, static_cast<__nv_bfloat16*>(out), ld_out,
+                  rows, cols, colmap, rowmap, st, device);
+  return gather(static_cast<const float*>(in), ld_in, in_rows, static_cast<float*>(out), ld_out, rows, cols, colmap,
+                rowmap, st, device);
+}
+
+cudaError_t scatter_dt(int32_t dt, const void* in, int64_t ld_in, void* out, int64_t ld_out, int64_t out_rows,
+                       int64_t rows, int cols, const int32_t* colmap, const int32_t* rowmap, cudaStream_t st,
+                       int device) {
+  if (dt == POETX_BF16)
+    return scatter(static_cast<const __nv_bfloat16*>(in), ld_in, static_cast<__nv_bfloat16*>(out), ld_out, out_rows,
+                   rows, cols, colmap, rowmap, st, device);
+  return scatter(static_cast<const float*>(in), ld_in, static_cast<float*>(out), ld_out, out_rows, rows, cols, colmap,
+                 rowmap, st, device);
+}
+
+// ---------------------------------------------------------------- GEMM descriptions
+// View of a [nblk][b][b] block array as a 2-D [nblk*b][b] matrix.
+Operand2D blocks_view(const void* p, int et, int nblk, int b, bool transposed) {
+  // transposed == false: element (mn, k) of block t is blk[t][k][mn] (MN-major)
+  // transposed == true : element (mn, k) of block t is blk[t][mn][k] (K-major)
+  Operand2D o;
+  o.ptr = p;
+  o.et = et;
+  o.rows = int64_t(nblk) * b;
+  o.cols = b;
+  o.ld = b;
+  o.mn_major = !transposed;
+  o.b_row = b;
+  o.b_col = 0;
+  return o;
+}
+
+// Row-major [rows][cols] activation whose column blocks of width b are the
+// batch (A operand of a block-diagonal product, K-major).
+Operand2D colblocks_view(const void* p, int et, int64_t rows, int64_t cols, int b) {
+  Operand2D o;
+  o.ptr = p;
+  o.et = et;
+  o.rows = rows;
+  o.cols = cols;
+  o.ld = cols;
+  o.mn_major = false;
+  o.b_row = 0;
+  o.b_col = b;
+  return o;
+}
+
+// out[:, jb:(j+1)b] = in[:, jb:(j+1)b] . op(G_j) for every block j.
+GemmDesc blockdiag_desc(const void* in, int et_in, int64_t T, int d, int b, const void* G, bool transpose_g,
+                        void* out, int et_out) {
+  GemmDesc g;
+  g.M = static_cast<int>(T);
+  g.N = b;
+  g.K = b;
+  g.batch = d / b;
+  g.A = colblocks_view(in, et_in, T, d, b);
+  // B(k, n) = G_j[k][n] (MN-major) or G_j[n][k] (K-major) for G_j^T.
+  g.B = blocks_view(G, et_in, d / b, b, transpose_g);
+  g.C.ptr = out;
+  g.C.et = et_out;
+  g.C.ld = d;
+  g.C.batch_stride = b;
+  return g;
+}
+
+// part[s][j] = (in1[:, jb:(j+1)b])^T in2[:, jb:(j+1)b] over token range s.
+GemmDesc blockgrad_desc(const void* in1, const void* in2, int et, int64_t T, int d, int b, int splits,
+                        float* part) {
+  GemmDesc g;
+  g.M = b;
+  g.N = b;
+  g.K = static_cast<int>(T);
+  g.batch = d / b;
+  g.splits = splits;
+  Operand2D a;
+  a.ptr = in1;
+  a.et = et;
+  a.rows = T;
+  a.cols = d;
+  a.ld = d;
+  a.mn_major = true;
+  a.b_row = 0;
+  a.b_col = b;
+  g.A = a;
+  Operand2D bo = a;
+  bo.ptr = in2;
+  g.B = bo;
+  g.C.ptr = part;
+  g.C.et = ET_F32;
+  g.C.ld = b;
+  g.C.batch_stride = int64_t(b) * b;
+  g.C.split_stride = int64_t(d / b) * b * b;
+  return g;
+}
+
+// Square b x b products over nblk blocks of fp32 scratch: C_t = opA(X_t) opB(Y_t).
+// opA: false -> X_t, true -> X_t^T.  opB: false -> Y_t, true -> Y_t^T.
+GemmDesc square_desc(const float* X, bool tA, const float* Y, bool tB, int nblk, int b, void* out, int et_out) {
+  GemmDesc g;
+  g.M = b;
+  g.N = b;
+  g.K = b;
+  g.batch = nblk;
+  // A(i, k) = X[i][k]  -> K-major view (row = i + t b, col = k)
+  // A(i, k) = X[k][i]  -> MN-major view (row = k + t b, col = i)
+  g.A = blocks_view(X, ET_F32, nblk, b, !tA);
+  // B(k, n) = Y[k][n]  -> MN-major;  B(k, n) = Y[n][k] -> K-major
+  g.B = blocks_view(Y, ET_F32, nblk, b, tB);
+  g.C.ptr = out;
+  g.C.et = et_out;
+  g.C.ld = b;
+  g.C.batch_stride = int64_t(b) * b;
+  return g;
+}
+
+AddDesc add_blocks(const float* p, int b, float beta) {
+  AddDesc a;
+  a.ptr = p;
+  a.ld = b;
+  a.batch_stride = int64_t(b) * b;
+  a.beta = beta;
+  return a;
+}
+
+// ---------------------------------------------------------------- CNP
+poetx_status cnp_build_impl(int32_t nblk, int32_t b, const float* q, int32_t dtype, void* G, Carver& ws,
+                            cudaStream_t st, int device) {
+  const size_t nbb = size_t(nblk) * b * b;
+  float* Q = ws.take<float>(sizeof(float) * nbb);
+  float* S = ws.take<float>(sizeof(float) * nbb);
+  float* H = ws.take<float>(sizeof(float) * nbb);
+  const bool tc_path = use_tc(dtype);
+  PROFILED(ST_CNP_ELEM, st, unpack_skew_kernel<<<static_cast<int>((int64_t(nblk) * b + 7) / 8), 256, 0, st>>>(q, nblk, b, Q));
+  POETX_CUDA(cudaGetLastError());
+  // S = Q Q
+  PROFILED(ST_CNP_GEMM, st, POETX_CUDA(launch_gemm(square_desc(Q, false, Q, false, nblk, b, S, ET_F32), tc_path, st, device)));
+  // H = 2Q + S
+  PROFILED(ST_CNP_ELEM, st, axpby_kernel<<<grid_for(nbb, 256, device), 256, 0, st>>>(Q, 2.f, S, 1.f, H, nbb));
+  POETX_CUDA(cudaGetLastError());
+  // G = H S + 2Q + 2S + I
+  GemmDesc g = square_desc(H, false, S, false, nblk, b, G, elem_type(dtype));
+  g.add1 = add_blocks(Q, b, 2.f);
+  g.add2 = add_blocks(S, b, 2.f);
+  g.diag = 1.f;
+  PROFILED(ST_CNP_GEMM, st, POETX_CUDA(launch_gemm(g, tc_path, st, device)));
+  return POETX_OK;
+}
+
+// dq from dG for G = I + 2A + 2S + H S with S = A A, H = 2A + S:
+//   dH = dG S^T;  dS = 2 dG + H^T dG + dH;  dA = 2 dG + 2 dH + dS A^T + A^T dS;
+//   dq_k = dA[i][j] - dA[j][i].
+poetx_status cnp_backward_impl(int32_t nblk, int32_t b, const float* q, const float* dG, float* dq,
+                               int32_t accumulate, int32_t dtype, Carver& ws, cudaStream_t st, int device) {
+  const size_t nbb = size_t(nblk) * b * b;
+  float* A = ws.take<float>(sizeof(float) * nbb);
+  float* S = ws.take<float>(sizeof(float) * nbb);
+  float* H = ws.take<float>(sizeof(float) * nbb);
+  float* dH = ws.take<float>(sizeof(float) * nbb);
+  float* dS = ws.take<float>(sizeof(float) * nbb);
+  float* T1 = ws.take<float>(sizeof(float) * nbb);
+  float* dA = ws.take<float>(sizeof(float) * nbb);
+  const bool tc_path = use_tc(dtype);
+  PROFILED(ST_CNP_ELEM, st, unpack_skew_kernel<<<static_cast<int>((int64_t(nblk) * b + 7) / 8), 256, 0, st>>>(q, nblk, b, A));
+  POETX_CUDA(cudaGetLastError());
+  PROFILED(ST_CNP_GEMM, st, POETX_CUDA(launch_gemm(square_desc(A, false, A, false, nblk, b, S, ET_F32), tc_path, st, device)));
+  PROFILED(ST_CNP_ELEM, st, axpby_kernel<<<grid_for(nbb, 256, device), 256, 0, st>>>(A, 2.f, S, 1.f, H, nbb));
+  POETX_CUDA(cudaGetLastError());
+  // dH = dG S^T
+  PROFILED(ST_CNP_GEMM, st, POETX_CUDA(launch_gemm(square_desc(dG, false, S, true, nblk, b, dH, ET_F32), tc_path, st, device)));
+  // dS = H^T dG + 2 dG + dH
+  {
+    GemmDesc g = square_desc(H, true, dG, false, nblk, b, dS, ET_F32);
+    g.add1 = add_blocks(dG, b, 2.f);
+    g.add2 = add_blocks(dH, b, 1.f);
+    PROFILED(ST_CNP_GEMM, st, POETX_CUDA(launch_gemm(g, tc_path, st, device)));
+  }
+  // T1 = dS A^T + 2 dG + 2 dH
+  {
+    GemmDesc g = square_desc(dS, false, A, true, nblk, b, T1, ET_F32);
+    g.add1 = add_blocks(dG, b, 2.f);
+    g.add2 = add_blocks(dH, b, 2.f);
+    PROFILED(ST_CNP_GEMM, st, POETX_CUDA(launch_gemm(g, tc_path, st, device)));
+  }
+  // dA = A^T dS + T1
+  {
+    GemmDesc g = square_desc(A, true, dS, false, nblk, b, dA, ET_F32);
+    g.add1 = add_blocks(T1, b, 1.f);
+    PROFILED(ST_CNP_GEMM, st, POETX_CUDA(launch_gemm(g, tc_path, st, device)));
+  }
+  PROFILED(ST_CNP_ELEM, st, fold_skew_kernel<<<static_cast<int>(int64_t(nblk) * b), 128, 0, st>>>(dA, nblk, b, dq, accumulate));
+  POETX_CUDA(cudaGetLastError());
+  return POETX_OK;
+}
+
+}  // namespace
+
+// ======================================================================== ABI
+
+extern "C" {
+
+const char* poetx_status_string(int status) {
+  switch (status) {
+    case POETX_OK: return "POETX_OK";
+    case POETX_E_ARG: return "POETX_E_ARG: null pointer, negative size or bad flag";
+    case POETX_E_SHAPE: return "POETX_E_SHAPE: b must divide m and n (and be a multiple of 64 for bf16)";
+    case POETX_E_DTYPE: return "POETX_E_DTYPE: unknown dtype";
+    case POETX_E_ALIGN: return "POETX_E_ALIGN: pointer not 16-byte aligned";
+    case POETX_E_WORKSPACE: return "POETX_E_WORKSPACE: workspace missing or too small";
+    case POETX_E_ARCH: return "POETX_E_ARCH: current device is not compute capability 10.0 (B200)";
+    case POETX_E_CUDA: return "POETX_E_CUDA: CUDA runtime error while queueing work";
+    default: return "POETX: unknown status";
+  }
+}
+
+int32_t poetx_version(void) { return 10000; }
+
+poetx_status poetx_device_error(uint32_t* code) {
+  if (!code) return POETX_E_ARG;
+  int dev;
+  POETX_TRY(current_device(&dev));
+  unsigned int v = 0, zero = 0;
+  POETX_CUDA(cudaDeviceSynchronize());
+  POETX_CUDA(cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v)));
+  POETX_CUDA(cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)));
+  *code = v;
+  return POETX_OK;
+}
+
+size_t poetx_cnp_workspace_bytes(int32_t nblk, int32_t b, int32_t dtype) {
+  (void)dtype;
+  if (nblk <= 0 || b < 2) return 0;
+  return kAlign + cnp_bwd_ws(nblk, b);
+}
+
+size_t poetx_forward_workspace_bytes(const poetx_layer* layer, int64_t T) {
+  if (check_layer(layer) != POETX_OK || T < 0) return 0;
+  return fwd_ws(layer, T);
+}
+
+size_t poetx_backward_workspace_bytes(const poetx_layer* layer, int64_t T) {
+  if (check_layer(layer) != POETX_OK || T < 0) return 0;
+  return bwd_ws(layer, T);
+}
+
+size_t poetx_merge_workspace_bytes(const poetx_layer* layer) {
+  if (check_layer(layer) != POETX_OK) return 0;
+  return merge_ws(layer);
+}
+
+size_t poetx_check_perm_workspace_bytes(int32_t len) {
+  if (len <= 0) return 0;
+  return kAlign + al(sizeof(int32_t) * size_t(len));
+}
+
+poetx_status poetx_frame_import(const poetx_layer* layer, const void* W0lin, void* stream) {
+  POETX_TRY(check_layer(layer));
+  POETX_TRY(check_ptr(W0lin));
+  int dev;
+  POETX_TRY(current_device(&dev));
+  const poetx_layer& L = *layer;
+  // W[j'][i'] = W0lin[permP[j']][permR[i']]
+  POETX_CUDA(gather_dt(L.dtype, W0lin, L.m, L.n, L.W, L.m, L.n, L.m, L.permR, L.permP,
+                       static_cast<cudaStream_t>(stream), dev));
+  return POETX_OK;
+}
+
+poetx_status poetx_frame_export(const poetx_layer* layer, void* W0lin, void* stream) {
+  POETX_TRY(check_layer(layer));
+  POETX_TRY(check_ptr(W0lin));
+  int dev;
+  POETX_TRY(current_device(&dev));
+  const poetx_layer& L = *layer;
+  // W0lin[permP[j']][permR[i']] = W[j'][i']
+  POETX_CUDA(scatter_dt(L.dtype, L.W, L.m, W0lin, L.m, L.n, L.n, L.m, L.permR, L.permP,
+                        static_cast<cudaStream_t>(stream), dev));
+  return POETX_OK;
+}
+
+poetx_status poetx_cnp_build(int32_t nblk, int32_t b, const float* q, int32_t dtype, void* G, void* ws,
+                             size_t ws_bytes, void* stream) {
+  POETX_TRY(check_dtype_b(dtype, b));
+  if (nblk < 0) return POETX_E_ARG;
+  if (nblk == 0) return POETX_OK;
+  POETX_TRY(check_ptr(q));
+  POETX_TRY(check_ptr(G));
+  if (!ws || ws_bytes < poetx_cnp_workspace_bytes(nblk, b, dtype)) return POETX_E_WORKSPACE;
+  int dev;
+  POETX_TRY(current_device(&dev));
+  Carver c(ws, ws_bytes);
+  return cnp_build_impl(nblk, b, q, dtype, G, c, static_cast<cudaStream_t>(stream), dev);
+}
+
+poetx_status poetx_cnp_backward(int32_t nblk, int32_t b, const float* q, const float* dG, float* dq,
+                                int32_t accumulate, int32_t dtype, void* ws, size_t ws_bytes, void* stream) {
+  POETX_TRY(check_dtype_b(dtype, b));
+  if (nblk < 0) return POETX_E_ARG;
+  if (nblk == 0) return POETX_OK;
+  POETX_TRY(check_ptr(q));
+  POETX_TRY(check_ptr(dG));
+  POETX_TRY(check_ptr(dq));
+  if (!ws || ws_bytes < poetx_cnp_workspace_bytes(nblk, b, dtype)) return POETX_E_WORKSPACE;
+  int dev;
+  POETX_TRY(current_device(&dev));
+  Carver c(ws, ws_bytes);
+  return cnp_backward_impl(nblk, b, q, dG, dq, accumulate, dtype, c, static_cast<cudaStream_t>(stream), dev);
+}
+
+poetx_status poetx_forward(const poetx_layer* layer, int64_t T, const void* x, void* z, void* y_save, void* ws,
+                           size_t ws_bytes, void* stream) {
+  POETX_TRY(check_layer(layer));
+  if (T < 0) return POETX_E_ARG;
+  if (T == 0) return POETX_OK;
+  POETX_TRY(check_ptr(x));
+  POETX_TRY(check_ptr(z));
+  if (y_save && !aligned16(y_save)) return POETX_E_ALIGN;
+  if (!ws || ws_bytes < fwd_ws(layer, T)) return POETX_E_WORKSPACE;
+  int dev;
+  POETX_TRY(current_device(&dev));
+  const poetx_layer& L = *layer;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int et = elem_type(L.dtype);
+  const size_t es = dtype_size(L.dtype);
+  const bool tc_path = use_tc(L.dtype);
+  Carver c(ws, ws_bytes);
+  void* Xg = c.take<uint8_t>(es * T * L.m);
+  void* U = c.take<uint8_t>(es * T * L.m);
+  void* V = c.take<uint8_t>(es * T * L.n);
+  void* Yw = c.take<uint8_t>(es * T * L.n);
+  void* Y = y_save ? y_save : Yw;
+  // Xg = x Psi_R^T  (columns gathered into the Psi_R frame)
+  PROFILED(ST_PERMUTE, st, POETX_CUDA(gather_dt(L.dtype, x, L.m, T, Xg, L.m, T, L.m, L.permR, nullptr, st, dev)));
+  // U_j = Xg_j G_Rj
+  PROFILED(ST_BLOCKDIAG, st, POETX_CUDA(launch_gemm(blockdiag_desc(Xg, et, T, L.m, L.b, L.GR, false, U, et), tc_path, st, dev)));
+  // Y = U W~  (W~ = Psi_R W0 Psi_P^T stored [n][m]: B(k=i', n=j') = W[j'][i'], K-major)
+  {
+    GemmDesc g;
+    g.M = static_cast<int>(T);
+    g.N = L.n;
+    g.K = L.m;
+    g.A = colblocks_view(U, et, T, L.m, 0);
+    Operand2D b;
+    b.ptr = L.W;
+    b.et = et;
+    b.rows = L.n;
+    b.cols = L.m;
+    b.ld = L.m;
+    b.mn_major = false;
+    g.B = b;
+    g.C.ptr = Y;
+    g.C.et = et;
+    g.C.ld = L.n;
+    PROFILED(ST_W0, st, POETX_CUDA(launch_gemm(g, tc_path, st, dev)));
+  }
+  // V_j = Y_j G_Pj
+  PROFILED(ST_BLOCKDIAG, st, POETX_CUDA(launch_gemm(blockdiag_desc(Y, et, T, L.n, L.b, L.GP, false, V, et), tc_path, st, dev)));
+  // z = V Psi_P  (columns scattered back to natural order)
+  PROFILED(ST_PERMUTE, st, POETX_CUDA(scatter_dt(L.dtype, V, L.n, z, L.n, T, T, L.n, L.permP, nullptr, st, dev)));
+  return POETX_OK;
+}
+
+poetx_status poetx_backward(const poetx_layer* layer, int64_t T, const void* x, const void* y_save,
+                            const void* dz, void* dx, float* dqR, float* dqP, int32_t accumulate, void* ws,
+                            size_t ws_bytes, void* stream) {
+  POETX_TRY(check_layer(layer));
+  if (T < 0) return POETX_E_ARG;
+  POETX_TRY(check_ptr(dqR));
+  POETX_TRY(check_ptr(dqP));
+  const poetx_layer& L = *layer;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int nR = L.m / L.b, nP = L.n / L.b;
+  const size_t triR = size_t(nR) * L.b * (L.b - 1) / 2, triP = size_t(nP) * L.b * (L.b - 1) / 2;
+  if (T == 0) {
+    if (!accumulate) {
+      POETX_CUDA(cudaMemsetAsync(dqR, 0, sizeof(float) * triR, st));
+      POETX_CUDA(cudaMemsetAsync(dqP, 0, sizeof(float) * triP, st));
+    }
+    return POETX_OK;
+  }
+  POETX_TRY(check_ptr(x));
+  POETX_TRY(check_ptr(y_save));
+  POETX_TRY(check_ptr(dz));
+  if (dx && !aligned16(dx)) return POETX_E_ALIGN;
+  if (!ws || ws_bytes < bwd_ws(layer, T)) return POETX_E_WORKSPACE;
+  int dev;
+  POETX_TRY(current_device(&dev));
+  const int et = elem_type(L.dtype);
+  const size_t es = dtype_size(L.dtype);
+  const bool tc_path = use_tc(L.dtype);
+  const int64_t mx = L.m > L.n ? L.m : L.n;
+  const size_t bb = size_t(L.b) * L.b;
+  const int sP = dg_splits(nP, L.b, T, L.dtype), sR = dg_splits(nR, L.b, T, L.dtype);
+  Carver c(ws, ws_bytes);
+  void* bufA = c.take<uint8_t>(es * T * mx);
+  void* bufB = c.take<uint8_t>(es * T * mx);
+  void* dU = c.take<uint8_t>(es * T * L.m);
+  float* partP = c.take<float>(sizeof(float) * sP * nP * bb);
+  float* partR = c.take<float>(sizeof(float) * sR * nR * bb);
+  float* dG = c.take<float>(sizeof(float) * (nR > nP ? nR : nP) * bb);
+
+  // dV = dz Psi_P^T
+  void* dV = bufA;
+  PROFILED(ST_PERMUTE, st, POETX_CUDA(gather_dt(L.dtype, dz, L.n, T, dV, L.n, T, L.n, L.permP, nullptr, st, dev)));
+  // dY_j = dV_j G_Pj^T
+  void* dY = bufB;
+  PROFILED(ST_BLOCKDIAG, st, POETX_CUDA(launch_gemm(blockdiag_desc(dV, et, T, L.n, L.b, L.GP, true, dY, et), tc_path, st, dev)));
+  // dG_Pj = Y_j^T dV_j (split over tokens)
+  PROFILED(ST_DG, st, POETX_CUDA(launch_gemm(blockgrad_desc(y_save, dV, et, T, L.n, L.b, sP, partP), tc_path, st, dev)));
+  // dU = dY W~^T  (B(k=j', n=i') = W[j'][i'], MN-major)
+  {
+    GemmDesc g;
+    g.M = static_cast<int>(T);
+    g.N = L.m;
+    g.K = L.n;
+    g.A = colblocks_view(dY, et, T, L.n, 0);
+    Operand2D b;
+    b.ptr = L.W;
+    b.et = et;
+    b.rows = L.n;
+    b.cols = L.m;
+    b.ld = L.m;
+    b.mn_major = true;
+    g.B = b;
+    g.C.ptr = dU;
+    g.C.et = et;
+    g.C.ld = L.m;
+    PROFILED(ST_W0, st, POETX_CUDA(launch_gemm(g, tc_path, st, dev)));
+  }
+  // Xg = x Psi_R^T (re-gathered; dV is dead)
+  void* Xg = bufA;
+  PROFILED(ST_PERMUTE, st, POETX_CUDA(gather_dt(L.dtype, x, L.m, T, Xg, L.m, T, L.m, L.permR, nullptr, st, dev)));
+  // dXg_j = dU_j G_Rj^T (dY is dead)
+  void* dXg = bufB;
+  if (dx) PROFILED(ST_BLOCKDIAG, st, POETX_CUDA(launch_gemm(blockdiag_desc(dU, et, T, L.m, L.b, L.GR, true, dXg, et), tc_path, st, dev)));
+  // dG_Rj = Xg_j^T dU_j
+  PROFILED(ST_DG, st, POETX_CUDA(launch_gemm(blockgrad_desc(Xg, dU, et, T, L.m, L.b, sR, partR), tc_path, st, dev)));
+  // dx = dXg Psi_R
+  if (dx) PROFILED(ST_PERMUTE, st, POETX_CUDA(scatter_dt(L.dtype, dXg, L.m, dx, L.m, T, T, L.m, L.permR, nullptr, st, dev)));
+  // dq from dG (fixed-order reduction of the token splits, then the CNP backward)
+  PROFILED(ST_REDUCE, st,
+           reduce_splits_kernel<<<grid_for(nP * bb / 4 + 1, 256, dev), 256, 0, st>>>(partP, sP, int64_t(nP) * bb, dG));
+  POETX_CUDA(cudaGetLastError());
+  {
+    Carver c2 = c;
+    POETX_TRY(cnp_backward_impl(nP, L.b, L.qP, dG, dqP, accumulate, L.dtype, c2, st, dev));
+  }
+  PROFILED(ST_REDUCE, st,
+           reduce_splits_kernel<<<grid_for(nR * bb / 4 + 1, 256, dev), 256, 0, st>>>(partR, sR, int64_t(nR) * bb, dG));
+  POETX_CUDA(cudaGetLastError());
+  {
+    Carver c2 = c;
+    POETX_TRY(cnp_backward_impl(nR, L.b, L.qR, dG, dqR, accumulate, L.dtype, c2, st, dev));
+  }
+  return POETX_OK;
+}
+
+poetx_status poetx_merge(const poetx_layer* layer, const int32_t* new_permR, const int32_t* new_permP,
+                         void* W_out, void* ws, size_t ws_bytes, void* stream) {
+  POETX_TRY(check_layer(layer));
+  POETX_TRY(check_ptr(new_permR));
+  POETX_TRY(check_ptr(new_permP));
+  POETX_TRY(check_ptr(W_out));
+  const poetx_layer& L = *layer;
+  const size_t es = dtype_size(L.dtype);
+  const size_t wbytes = es * size_t(L.n) * L.m;
+  {
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(L.W), b0 = reinterpret_cast<uintptr_t>(W_out);
+    if (a0 < b0 + wbytes && b0 < a0 + wbytes) return POETX_E_ARG;
+  }
+  if (!ws || ws_bytes < merge_ws(layer)) return POETX_E_WORKSPACE;
+  int dev;
+  POETX_TRY(current_device(&dev));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int et = elem_type(L.dtype);
+  const bool tc_path = use_tc(L.dtype);
+  const int nR = L.m / L.b, nP = L.n / L.b;
+  const size_t nm = size_t(L.n) * L.m;
+  Carver c(ws, ws_bytes);
+  float* B1 = c.take<float>(sizeof(float) * nm);
+  float* At = c.take<float>(sizeof(float) * nm);
+  float* GPf = c.take<float>(sizeof(float) * size_t(nP) * L.b * L.b);
+  int32_t* invR = c.take<int32_t>(sizeof(int32_t) * L.m);
+  int32_t* invP = c.take<int32_t>(sizeof(int32_t) * L.n);
+  int32_t* sigR = c.take<int32_t>(sizeof(int32_t) * L.m);
+  int32_t* sigP = c.take<int32_t>(sizeof(int32_t) * L.n);
+
+  // Stored W~ = (Psi_R W0 Psi_P^T)^T.  New weight R W0 P in the old frame is
+  // A' = Diag(G_R) W~ Diag(G_P), stored transposed:
+  //   At = Diag(G_P)^T . W . Diag(G_R)^T     ([n][m])
+  // pass 1: B1 = W . Diag(G_R)^T  (column blocks i: B1[:, ib:] = W[:, ib:] G_Ri^T)
+  {
+    GemmDesc g;
+    g.M = L.n;
+    g.N = L.b;
+    g.K = L.b;
+    g.batch = nR;
+    g.A = colblocks_view(L.W, et, L.n, L.m, L.b);
+    g.B = blocks_view(L.GR, et, nR, L.b, true);
+    g.C.ptr = B1;
+    g.C.et = ET_F32;
+    g.C.ld = L.m;
+    g.C.batch_stride = L.b;
+    PROFILED(ST_MERGE, st, POETX_CUDA(launch_gemm(g, tc_path, st, dev)));
+  }
+  // pass 2: At[jb:(j+1)b, :] = G_Pj^T . B1[jb:(j+1)b, :]
+  {
+    const float* GPsrc;
+    if (L.dtype == POETX_BF16) {
+      const int64_t cnt = int64_t(nP) * L.b * L.b;
+      bf16_to_f32_kernel<<<grid_for(cnt, 256, dev), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(L.GP), GPf, cnt);
+      POETX_CUDA(cudaGetLastError());
+      GPsrc = GPf;
+    } else {
+      GPsrc = static_cast<const float*>(L.GP);
+    }
+    GemmDesc g;
+    g.M = L.b;
+    g.N = L.m;
+    g.K = L.b;
+    g.batch = nP;
+    // A(r, k) = G_Pj[k][r]: MN-major view of the blocks
+    g.A = blocks_view(GPsrc, ET_F32, nP, L.b, false);
+    // B(k, c) = B1[jb + k][c]: MN-major view, batch moves down b rows
+    Operand2D b;
+    b.ptr = B1;
+    b.et = ET_F32;
+    b.rows = L.n;
+    b.cols = L.m;
+    b.ld = L.m;
+    b.mn_major = true;
+    b.b_row = L.b;
+    b.b_col = 0;
+    g.B = b;
+    g.C.ptr = At;
+    g.C.et = ET_F32;
+    g.C.ld = L.m;
+    g.C.batch_stride = int64_t(L.b) * L.m;
+    PROFILED(ST_MERGE, st, POETX_CUDA(launch_gemm(g, tc_path, st, dev)));
+  }
+  // New frame: W'[j'][i'] = At[sigP[j']][sigR[i']], sig = perm_old^-1 o perm_new.
+  invert_perm_kernel<<<(L.m + 255) / 256, 256, 0, st>>>(L.permR, invR, L.m);
+  invert_perm_kernel<<<(L.n + 255) / 256, 256, 0, st>>>(L.permP, invP, L.n);
+  compose_perm_kernel<<<(L.m + 255) / 256, 256, 0, st>>>(invR, new_permR, sigR, L.m);
+  compose_perm_kernel<<<(L.n + 255) / 256, 256, 0, st>>>(invP, new_permP, sigP, L.n);
+  POETX_CUDA(cudaGetLastError());
+  if (L.dtype == POETX_BF16)
+    POETX_CUDA(gather(static_cast<const float*>(At), L.m, L.n, static_cast<__nv_bfloat16*>(W_out), L.m, L.n, L.m,
+                      sigR, sigP, st, dev));
+  else
+    POETX_CUDA(gather(static_cast<const float*>(At), L.m, L.n, static_cast<float*>(W_out), L.m, L.n, L.m, sigR, sigP,
+                      st, dev));
+  // Reset: Q = 0, G = I.
+  POETX_CUDA(cudaMemsetAsync(L.qR, 0, sizeof(float) * size_t(nR) * L.b * (L.b - 1) / 2, st));
+  POETX_CUDA(cudaMemsetAsync(L.qP, 0, sizeof(float) * size_t(nP) * L.b * (L.b - 1) / 2, st));
+  const int64_t cR = int64_t(nR) * L.b * L.b, cP = int64_t(nP) * L.b * L.b;
+  if (L.dtype == POETX_BF16) {
+    identity_blocks_kernel<__nv_bfloat16>
+        <<<grid_for(cR, 256, dev), 256, 0, st>>>(static_cast<__nv_bfloat16*>(L.GR), nR, L.b);
+    identity_blocks_kernel<__nv_bfloat16>
+        <<<grid_for(cP, 256, dev), 256, 0, st>>>(static_cast<__nv_bfloat16*>(L.GP), nP, L.b);
+  } else {
+    identity_blocks_kernel<float><<<grid_for(cR, 256, dev), 256, 0, st>>>(static_cast<float*>(L.GR), nR, L.b);
+    identity_blocks_kernel<float><<<grid_for(cP, 256, dev), 256, 0, st>>>(static_cast<float*>(L.GP), nP, L.b);
+  }
+  POETX_CUDA(cudaGetLastError());
+  return POETX_OK;
+}
+
+poetx_status poetx_check_perm(const int32_t* perm, int32_t len, int32_t* d_ok, void* ws, size_t ws_bytes,
+                              void* stream) {
+  if (len <= 0) return POETX_E_ARG;
+  POETX_TRY(check_ptr(perm));
+  if (!d_ok) return POETX_E_ARG;
+  if (!ws || ws_bytes < poetx_check_perm_workspace_bytes(len)) return POETX_E_WORKSPACE;
+  int dev;
+  POETX_TRY(current_device(&dev));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Carver c(ws, ws_bytes);
+  int32_t* hist = c.take<int32_t>(sizeof(int32_t) * len);
+  POETX_CUDA(cudaMemsetAsync(hist, 0, sizeof(int32_t) * len, st));
+  set_int_kernel<<<1, 1, 0, st>>>(d_ok, 1);
+  perm_histogram_kernel<<<(len + 255) / 256, 256, 0, st>>>(perm, hist, len, d_ok);
+  perm_check_kernel<<<(len + 255) / 256, 256, 0, st>>>(hist, len, d_ok);
+  POETX_CUDA(cudaGetLastError());
+  return POETX_OK;
+}
+
+int32_t poetx_profile_stage_count(void) { return ST_COUNT; }
+
+const char* poetx_profile_stage_name(int32_t stage) {
+  if (stage < 0 || stage >= ST_COUNT) return "unknown";
+  return kStageNames[stage];
+}
+
+poetx_status poetx_profile_begin(void) {
+  Profiler& P = profiler();
+  std::lock_guard<std::mutex> g(P.mu);
+  P.on = true;
+  P.used = 0;
+  P.recs.clear();
+  return POETX_OK;
+}
+
+poetx_status poetx_profile_end(double* ms_per_stage, int64_t* launches_per_stage, int32_t nstages) {
+  if (!ms_per_stage || !launches_per_stage || nstages < 0) return POETX_E_ARG;
+  Profiler& P = profiler();
+  std::lock_guard<std::mutex> g(P.mu);
+  for (int i = 0; i < nstages; ++i) {
+    ms_per_stage[i] = 0.0;
+    launches_per_stage[i] = 0;
+  }
+  poetx_status st = POETX_OK;
+  for (const auto& r : P.recs) {
+    if (cudaEventSynchronize(P.pool[r.second + 1]) != cudaSuccess) {
+      (void)cudaGetLastError();
+      st = POETX_E_CUDA;
+      break;
+    }
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, P.pool[r.second], P.pool[r.second + 1]) != cudaSuccess) {
+      (void)cudaGetLastError();
+      st = POETX_E_CUDA;
+      break;
+    }
+    if (r.first < nstages) {
+      ms_per_stage[r.first] += ms;
+      launches_per_stage[r.first] += 1;
+    }
+  }
+  P.on = false;
+  P.used = 0;
+  P.recs.clear();
+  return st;
+}
+
+}  // extern "C"

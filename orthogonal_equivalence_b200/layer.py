@@ -1,0 +1,123 @@
+"""PoetxLinear: device buffers of one POET-X layer and thin wrappers around
+the C calls (allocation with torch, arithmetic in libpoetx.so).
+
+State of a layer (POET-X write-up, sections 2-3 and the merge step of its API
+snippet): the frozen weight stored in the frame of the current permutations
+(W[j'][i'] = W0[permR[i']][permP[j']], [n][m]), the permutations, the packed
+triangles qR, qP (the trainable parameters) and the G blocks built from them.
+"""
+from __future__ import annotations
+
+from typing import Optional, Tuple
+
+import torch
+
+from . import (POETX_BF16, POETX_FP32, make_layer, poetx_backward, poetx_backward_workspace_bytes,
+               poetx_cnp_build, poetx_cnp_workspace_bytes, poetx_forward, poetx_forward_workspace_bytes,
+               poetx_frame_export, poetx_frame_import, poetx_merge, poetx_merge_workspace_bytes)
+
+_TORCH_DTYPE = {POETX_BF16: torch.bfloat16, POETX_FP32: torch.float32}
+
+
+class PoetxLinear:
+    """One layer z = x R W0 P (x: [T][m], z: [T][n])."""
+
+    def __init__(self, m: int, n: int, b: int, dtype: int, device="cuda"):
+        if dtype not in _TORCH_DTYPE:
+            raise ValueError("dtype must be POETX_BF16 or POETX_FP32")
+        self.m, self.n, self.b, self.dtype = m, n, b, dtype
+        self.device = torch.device(device)
+        td = _TORCH_DTYPE[dtype]
+        tri = b * (b - 1) // 2
+        self.W = torch.empty((n, m), dtype=td, device=self.device)
+        self.permR = torch.empty(m, dtype=torch.int32, device=self.device)
+        self.permP = torch.empty(n, dtype=torch.int32, device=self.device)
+        self.qR = torch.zeros((m // b, tri), dtype=torch.float32, device=self.device)
+        self.qP = torch.zeros((n // b, tri), dtype=torch.float32, device=self.device)
+        self.GR = torch.empty((m // b, b, b), dtype=td, device=self.device)
+        self.GP = torch.empty((n // b, b, b), dtype=td, device=self.device)
+        self._ws = {}
+
+    @property
+    def torch_dtype(self) -> torch.dtype:
+        return _TORCH_DTYPE[self.dtype]
+
+    def abi(self):
+        return make_layer(self.m, self.n, self.b, self.dtype, self.W, self.permR, self.permP, self.qR, self.qP,
+                          self.GR, self.GP)
+
+    def workspace(self, kind: str, nbytes: int) -> torch.Tensor:
+        ws = self._ws.get(kind)
+        if ws is None or ws.numel() < nbytes:
+            ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=self.device)
+            self._ws[kind] = ws
+        return ws
+
+    # -------------------------------------------------------------- state
+    def load(self, W0lin: torch.Tensor, permR: torch.Tensor, permP: torch.Tensor, qR: torch.Tensor,
+             qP: torch.Tensor, stream=None) -> None:
+        """Set the permutations and triangles, import the natural nn.Linear
+        weight W0^T ([n][m]) into the frame, and build G."""
+        self.permR.copy_(permR)
+        self.permP.copy_(permP)
+        self.qR.copy_(qR)
+        self.qP.copy_(qP)
+        poetx_frame_import(self.abi(), W0lin.contiguous(), stream)
+        self.build(stream)
+
+    def export_weight(self, stream=None) -> torch.Tensor:
+        out = torch.empty((self.n, self.m), dtype=self.torch_dtype, device=self.device)
+        poetx_frame_export(self.abi(), out, stream)
+        return out
+
+    def build(self, stream=None) -> None:
+        """G_R, G_P from qR, qP (Cayley-Neumann)."""
+        nR, nP = self.m // self.b, self.n // self.b
+        nb = poetx_cnp_workspace_bytes(max(nR, nP), self.b, self.dtype)
+        ws = self.workspace("cnp", nb)
+        poetx_cnp_build(nR, self.b, self.qR, self.dtype, self.GR, ws, nb, stream)
+        poetx_cnp_build(nP, self.b, self.qP, self.dtype, self.GP, ws, nb, stream)
+
+    # -------------------------------------------------------------- layer
+    def forward(self, x: torch.Tensor, save: bool = True, z: Optional[torch.Tensor] = None,
+                y: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+        T = x.shape[0]
+        if z is None:
+            z = torch.empty((T, self.n), dtype=self.torch_dtype, device=self.device)
+        if save and y is None:
+            y = torch.empty((T, self.n), dtype=self.torch_dtype, device=self.device)
+        L = self.abi()
+        nb = poetx_forward_workspace_bytes(L, T)
+        ws = self.workspace("fwd", nb)
+        poetx_forward(L, T, x, z, y if save else None, ws, nb, stream)
+        return z, (y if save else None)
+
+    def backward(self, x: torch.Tensor, y: torch.Tensor, dz: torch.Tensor, need_dx: bool = True,
+                 dx: Optional[torch.Tensor] = None, dqR: Optional[torch.Tensor] = None,
+                 dqP: Optional[torch.Tensor] = None, accumulate: bool = False, stream=None):
+        T = x.shape[0]
+        if need_dx and dx is None:
+            dx = torch.empty((T, self.m), dtype=self.torch_dtype, device=self.device)
+        if dqR is None:
+            dqR = torch.empty_like(self.qR)
+        if dqP is None:
+            dqP = torch.empty_like(self.qP)
+        L = self.abi()
+        nb = poetx_backward_workspace_bytes(L, T)
+        ws = self.workspace("bwd", nb)
+        poetx_backward(L, T, x, y, dz, dx if need_dx else None, dqR, dqP, int(accumulate), ws, nb, stream)
+        return (dx if need_dx else None), dqR, dqP
+
+    def merge(self, new_permR: torch.Tensor, new_permP: torch.Tensor, stream=None) -> None:
+        """W0 <- R W0 P, re-expressed in the frame of the new permutations;
+        q = 0 and G = I afterwards."""
+        L = self.abi()
+        nb = poetx_merge_workspace_bytes(L)
+        ws = self.workspace("merge", nb)
+        W_out = torch.empty_like(self.W)
+        newR = new_permR.to(device=self.device, dtype=torch.int32).contiguous()
+        newP = new_permP.to(device=self.device, dtype=torch.int32).contiguous()
+        poetx_merge(L, newR, newP, W_out, ws, nb, stream)
+        self.W = W_out
+        self.permR.copy_(newR)
+        self.permP.copy_(newP)

@@ -1,0 +1,103 @@
+"""CPU checks of the C ABI: libpoetx.so loads, exports every function that
+include/poetx.h declares, and rejects bad arguments before touching a device.
+No compute call is made here (this host has no GPU)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import orthogonal_equivalence_b200 as px
+from orthogonal_equivalence_b200 import build as pbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    pbuild.build()
+    return px.lib()
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "poetx.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(poetx_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_expected_calls():
+    names = header_functions()
+    for want in ["poetx_cnp_build", "poetx_cnp_backward", "poetx_forward", "poetx_backward", "poetx_merge",
+                 "poetx_frame_import", "poetx_frame_export"]:
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", px.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (poetx_\w+)", out))
+    missing = [n for n in header_functions() if n not in exported]
+    assert not missing, missing
+    for n in header_functions():
+        assert hasattr(lib, n)
+    assert set(px.SIGNATURES) == set(header_functions())
+
+
+def test_status_strings(lib):
+    for code, name in px.STATUS_NAMES.items():
+        assert px.poetx_status_string(code).startswith(name)
+    assert "unknown" in px.poetx_status_string(99)
+    assert px.poetx_version() == 10000
+
+
+def _layer(m=512, n=256, b=64, dtype=px.POETX_BF16, ptr=4096):
+    return px.poetx_layer(m, n, b, dtype, ptr, ptr, ptr, ptr, ptr, ptr, ptr)
+
+
+def test_workspace_sizes_are_host_arithmetic(lib):
+    L = _layer()
+    T = 300
+    assert px.poetx_forward_workspace_bytes(L, T) >= 2 * T * (2 * 512 + 2 * 256)
+    assert px.poetx_backward_workspace_bytes(L, T) >= 2 * T * (2 * 512 + 512)
+    assert px.poetx_merge_workspace_bytes(L) >= 2 * 4 * 512 * 256
+    assert px.poetx_cnp_workspace_bytes(8, 64, px.POETX_BF16) >= 7 * 4 * 8 * 64 * 64
+    assert px.poetx_check_perm_workspace_bytes(100) >= 400
+    # invalid layers size to 0
+    assert px.poetx_forward_workspace_bytes(_layer(b=48), T) == 0   # bf16 needs b % 64 == 0
+    assert px.poetx_forward_workspace_bytes(_layer(m=500), T) == 0  # b must divide m
+    assert px.poetx_forward_workspace_bytes(_layer(dtype=7), T) == 0
+
+
+def test_validation_before_any_launch(lib):
+    # every rejected call returns its status without touching a device
+    assert lib.poetx_forward(None, 10, 4096, 4096, None, 4096, 1 << 30, None) == 1          # E_ARG
+    L = _layer(m=500)
+    assert lib.poetx_forward(ctypes.byref(L), 10, 4096, 4096, None, 4096, 1 << 30, None) == 2  # E_SHAPE
+    L = _layer(dtype=5)
+    assert lib.poetx_forward(ctypes.byref(L), 10, 4096, 4096, None, 4096, 1 << 30, None) == 3  # E_DTYPE
+    L = _layer(ptr=4100)
+    assert lib.poetx_forward(ctypes.byref(L), 10, 4096, 4096, None, 4096, 1 << 30, None) == 4  # E_ALIGN
+    L = _layer()
+    assert lib.poetx_forward(ctypes.byref(L), -1, 4096, 4096, None, 4096, 1 << 30, None) == 1  # T < 0
+    assert lib.poetx_forward(ctypes.byref(L), 10, 4096, 4096, None, 4096, 16, None) == 5       # ws small
+    assert lib.poetx_forward(ctypes.byref(L), 10, None, 4096, None, 4096, 1 << 30, None) == 1  # x NULL
+    assert lib.poetx_backward(ctypes.byref(L), 10, 4096, None, 4096, None, 4096, 4096, 0, 4096, 1 << 30,
+                              None) == 1                                                      # y_save NULL
+    assert lib.poetx_cnp_build(4, 48, 4096, px.POETX_BF16, 4096, 4096, 1 << 30, None) == 2    # b % 64
+    assert lib.poetx_cnp_build(4, 64, 4096, 9, 4096, 4096, 1 << 30, None) == 3
+    assert lib.poetx_cnp_build(4, 64, 4096, px.POETX_BF16, 4096, 4096, 8, None) == 5
+    assert lib.poetx_cnp_backward(4, 1, 4096, 4096, 4096, 0, px.POETX_FP32, 4096, 1 << 30, None) == 2
+    # merge output may not overlap the stored weight
+    assert lib.poetx_merge(ctypes.byref(L), 4096, 4096, 4096, 4096, 1 << 30, None) == 1
+    assert lib.poetx_check_perm(4096, 0, 4096, 4096, 1 << 20, None) == 1
+
+
+def test_no_device_call_fails_cleanly(lib):
+    # a fully valid call on a host without a GPU reports a CUDA error, not a crash
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("host has a GPU")
+    L = _layer()
+    T = 10
+    ws = px.poetx_forward_workspace_bytes(L, T)
+    assert lib.poetx_forward(ctypes.byref(L), T, 4096, 4096, 4096, 4096, ws, None) == 7

@@ -1,0 +1,269 @@
+"""GPU parity of libpoetx.so against the float64 oracle on the same seeded
+inputs (POET-X write-up, sections 1-3 and the merge step).
+
+Bars: permutation / frame / index work bit-exact; fp32 layers normwise max
+error <= 1e-5; bf16 layers relative Frobenius error <= 1e-2 on z, dx, dqR, dqP
+and the merged weight.  Reduced shapes keep every recipe of the workloads but
+span several tiles with ragged token tails; the full-size workloads are
+checked on sampled token rows and sampled blocks, in the launch configuration
+the benchmark uses."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import orthogonal_equivalence_b200 as px
+import poetx_inputs as pi
+from orthogonal_equivalence_b200 import build as pbuild
+
+from gpu_util import bits, check, dev, host64, make_layer, poetx_dtype
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def library():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    pbuild.build()
+    px.lib()
+    px.poetx_device_error()  # clear
+    yield
+    torch.cuda.synchronize()
+    assert px.poetx_device_error() == 0, "a kernel recorded a device error (timeout or bad index)"
+
+
+# (workload recipe, m, n, b, T); None = the workload's own size
+SMALL = [
+    ("tiny", None, None, None, None),
+    ("tiny", 192, 320, 64, 77),
+    ("attn3b", 512, 512, 256, 300),
+    ("up8b", 512, 1792, 256, 200),
+    ("down13b", 1536, 1024, 512, 130),
+    ("block8b", 1024, 256, 256, 257),
+    ("block8b", 256, 768, 256, 1),
+]
+
+
+def _inputs(name, m, n, b, T, layer=0, **kw):
+    return pi.layer_inputs(pi.CONFIGS[name], layer=layer, T=T, m=m, n=n, b=b, **kw)
+
+
+def _oracle_all(inp):
+    W0 = inp.W0lin64.T
+    GR = oracle.cnp_blocks(inp.qR, inp.b)
+    GP = oracle.cnp_blocks(inp.qP, inp.b)
+    z = oracle.forward(inp.x64, W0, inp.permR, GR, inp.permP, GP)
+    dX, dGR, dGP = oracle.backward(inp.x64, W0, inp.permR, GR, inp.permP, GP, inp.dz64)
+    return z, dX, oracle.cnp_backward(inp.qR, inp.b, dGR), oracle.cnp_backward(inp.qP, inp.b, dGP), GR, GP
+
+
+def _run(L, inp):
+    x = dev(inp.x, inp.dtype)
+    dz = dev(inp.dz, inp.dtype)
+    z, y = L.forward(x)
+    dx, dqR, dqP = L.backward(x, y, dz)
+    torch.cuda.synchronize()
+    return z, y, dx, dqR, dqP
+
+
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: "-".join(str(v) for v in c))
+def test_layer_forward_backward_parity(case):
+    inp = _inputs(*case)
+    L = make_layer(inp)
+    z, _, dx, dqR, dqP = _run(L, inp)
+    zo, dxo, dqRo, dqPo, _, _ = _oracle_all(inp)
+    check(host64(z), zo, inp.dtype, "z")
+    check(host64(dx), dxo, inp.dtype, "dx")
+    check(host64(dqR), dqRo, inp.dtype, "dqR")
+    check(host64(dqP), dqPo, inp.dtype, "dqP")
+
+
+@pytest.mark.parametrize("dtype,b,nblk", [("fp32", 64, 8), ("bf16", 256, 5), ("bf16", 512, 3), ("bf16", 64, 9),
+                                          ("fp32", 6, 4)])
+def test_cnp_build_and_backward_parity(dtype, b, nblk):
+    g = np.random.Generator(np.random.PCG64(1000 + b + nblk))
+    q = (g.standard_normal((nblk, b * (b - 1) // 2)) * 0.01).astype(np.float32)
+    dG = g.standard_normal((nblk, b, b)).astype(np.float32)
+    pd = poetx_dtype(dtype)
+    td = torch.bfloat16 if dtype == "bf16" else torch.float32
+    qd = torch.from_numpy(q).cuda()
+    G = torch.empty((nblk, b, b), dtype=td, device="cuda")
+    nb = px.poetx_cnp_workspace_bytes(nblk, b, pd)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    px.poetx_cnp_build(nblk, b, qd, pd, G, ws, nb)
+    dq = torch.empty_like(qd)
+    px.poetx_cnp_backward(nblk, b, qd, torch.from_numpy(dG).cuda(), dq, 0, pd, ws, nb)
+    torch.cuda.synchronize()
+    Go = oracle.cnp_blocks(q, b)
+    dqo = oracle.cnp_backward(q, b, dG.astype(np.float64))
+    check(host64(G), Go, dtype, "G")
+    check(host64(dq), dqo, dtype, "dq")
+    # accumulate adds onto what is there
+    px.poetx_cnp_backward(nblk, b, qd, torch.from_numpy(dG).cuda(), dq, 1, pd, ws, nb)
+    torch.cuda.synchronize()
+    check(host64(dq), 2 * dqo, dtype, "dq accumulated")
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_zero_q_gives_identity_and_plain_linear(dtype):
+    name = "tiny" if dtype == "fp32" else "attn3b"
+    b = 64 if dtype == "fp32" else 256
+    inp = _inputs(name, 512, 768, b, 150, zero_q=True)
+    L = make_layer(inp)
+    eye = np.broadcast_to(np.eye(b), (512 // b, b, b))
+    assert np.array_equal(host64(L.GR), eye)
+    assert np.array_equal(host64(L.GP), np.broadcast_to(np.eye(b), (768 // b, b, b)))
+    z, _ = L.forward(dev(inp.x, dtype))
+    torch.cuda.synchronize()
+    check(host64(z), inp.x64 @ inp.W0lin64.T, dtype, "z with Q = 0")
+
+
+@pytest.mark.parametrize("dtype,m,n", [("fp32", 192, 320), ("bf16", 1024, 768), ("bf16", 14336, 256)])
+def test_frame_import_export_bit_exact(dtype, m, n):
+    name = "tiny" if dtype == "fp32" else "block8b"
+    inp = _inputs(name, m, n, 64, 4)
+    L = make_layer(inp)
+    torch.cuda.synchronize()
+    want = oracle.to_frame(inp.W0lin, inp.permR, inp.permP)
+    assert np.array_equal(bits(L.W), want.view(np.uint16 if dtype == "bf16" else np.uint32))
+    back = L.export_weight()
+    torch.cuda.synchronize()
+    assert np.array_equal(bits(back), inp.W0lin.view(np.uint16 if dtype == "bf16" else np.uint32))
+
+
+def _merge_check(inp, merge_index=1):
+    L = make_layer(inp)
+    x = dev(inp.x, inp.dtype)
+    z_before, _ = L.forward(x, save=False)
+    newR, newP = pi.merge_perms(pi.CONFIGS["tiny"] if inp.dtype == "fp32" else pi.CONFIGS["down13b"], 0,
+                                merge_index, inp.m, inp.n)
+    L.merge(torch.from_numpy(newR).cuda(), torch.from_numpy(newP).cuda())
+    W_nat = L.export_weight()
+    torch.cuda.synchronize()
+    GR = oracle.cnp_blocks(inp.qR, inp.b)
+    GP = oracle.cnp_blocks(inp.qP, inp.b)
+    W_o = oracle.merge(inp.W0lin64.T, inp.permR, GR, inp.permP, GP)   # natural m x n
+    check(host64(W_nat), W_o.T, inp.dtype, "merged weight")
+    assert not np.any(host64(L.qR)) and not np.any(host64(L.qP))
+    assert np.array_equal(host64(L.GR), np.broadcast_to(np.eye(inp.b), L.GR.shape))
+    assert np.array_equal(bits(L.permR), newR.view(np.uint32))
+    # function preservation: same z before and after the merge
+    z_after, _ = L.forward(x, save=False)
+    torch.cuda.synchronize()
+    check(host64(z_after), host64(z_before), inp.dtype, "z after merge")
+    return L
+
+
+@pytest.mark.parametrize("case", [("tiny", None, None, None, 64), ("down13b", 1536, 1024, 512, 64),
+                                  ("attn3b", 768, 512, 256, 33)], ids=lambda c: c[0])
+def test_merge_parity(case):
+    _merge_check(_inputs(*case))
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_merge_with_zero_q_is_exact_reframing(dtype):
+    name = "tiny" if dtype == "fp32" else "attn3b"
+    b = 64 if dtype == "fp32" else 256
+    inp = _inputs(name, 512, 768, b, 8, zero_q=True)
+    L = make_layer(inp)
+    newR, newP = pi.merge_perms(pi.CONFIGS[name], 0, 1, 512, 768)
+    L.merge(torch.from_numpy(newR).cuda(), torch.from_numpy(newP).cuda())
+    torch.cuda.synchronize()
+    want = oracle.to_frame(inp.W0lin, newR, newP)
+    assert np.array_equal(bits(L.W), want.view(np.uint16 if dtype == "bf16" else np.uint32))
+
+
+def test_empty_and_single_token():
+    inp = _inputs("attn3b", 512, 512, 256, 1)
+    L = make_layer(inp)
+    x = dev(inp.x, "bf16")
+    z = torch.empty((0, 512), dtype=torch.bfloat16, device="cuda")
+    L.forward(x[:0], z=z)          # T = 0: no-op
+    dqR = torch.full_like(L.qR, 7.0)
+    dqP = torch.full_like(L.qP, 7.0)
+    L.backward(x[:0], z, z, need_dx=True, dx=torch.empty((0, 512), dtype=torch.bfloat16, device="cuda"),
+               dqR=dqR, dqP=dqP)
+    torch.cuda.synchronize()
+    assert not torch.any(dqR) and not torch.any(dqP)
+    z1, _, dx1, dqR1, dqP1 = _run(L, inp)
+    zo, dxo, dqRo, dqPo, _, _ = _oracle_all(inp)
+    check(host64(z1), zo, "bf16", "z T=1")
+    check(host64(dx1), dxo, "bf16", "dx T=1")
+    check(host64(dqR1), dqRo, "bf16", "dqR T=1")
+
+
+def test_backward_is_deterministic_and_accumulates():
+    inp = _inputs("up8b", 512, 1024, 256, 700)
+    L = make_layer(inp)
+    x, dz = dev(inp.x, "bf16"), dev(inp.dz, "bf16")
+    _, y = L.forward(x)
+    _, a_R, a_P = L.backward(x, y, dz)
+    _, b_R, b_P = L.backward(x, y, dz)
+    torch.cuda.synchronize()
+    assert np.array_equal(bits(a_R), bits(b_R)) and np.array_equal(bits(a_P), bits(b_P))
+    acc_R, acc_P = a_R.clone(), a_P.clone()
+    L.backward(x, y, dz, need_dx=False, dqR=acc_R, dqP=acc_P, accumulate=True)
+    torch.cuda.synchronize()
+    np.testing.assert_allclose(host64(acc_R), 2 * host64(a_R), rtol=1e-6, atol=0)
+
+
+def test_check_perm_and_errors():
+    n = 1000
+    perm = torch.from_numpy(pi.permutation(5, n)).cuda()
+    ok = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nb = px.poetx_check_perm_workspace_bytes(n)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    px.poetx_check_perm(perm, n, ok, ws, nb)
+    torch.cuda.synchronize()
+    assert ok.item() == 1
+    bad = perm.clone()
+    bad[3] = bad[4]
+    px.poetx_check_perm(bad, n, ok, ws, nb)
+    torch.cuda.synchronize()
+    assert ok.item() == 0
+    bad[3] = n + 5
+    px.poetx_check_perm(bad, n, ok, ws, nb)
+    torch.cuda.synchronize()
+    assert ok.item() == 0
+    # a workspace that is too small is refused before anything is queued
+    inp = _inputs("attn3b", 512, 512, 256, 16)
+    L = make_layer(inp)
+    with pytest.raises(px.PoetxError) as e:
+        px.poetx_forward(L.abi(), 16, dev(inp.x, "bf16"), torch.empty((16, 512), dtype=torch.bfloat16,
+                                                                       device="cuda"), None, ws, 64)
+    assert e.value.status == 5
+
+
+# ------------------------------------------------------------------ full-size workloads
+FULL = ["attn3b", "up8b", "down13b", "block8b"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_sampled_parity(name):
+    cfg = pi.CONFIGS[name]
+    for layer in range(len(cfg.layers)):
+        inp = pi.layer_inputs(cfg, layer)
+        L = make_layer(inp)
+        z, _, dx, dqR, dqP = _run(L, inp)
+        rows = pi.random_token_rows(7 + layer, inp.T, 48)
+        W0 = inp.W0lin64.T
+        GR = oracle.cnp_blocks(inp.qR, inp.b)
+        GP = oracle.cnp_blocks(inp.qP, inp.b)
+        zo = oracle.forward(inp.x64[rows], W0, inp.permR, GR, inp.permP, GP)
+        dxo, _, _ = oracle.backward(inp.x64[rows], W0, inp.permR, GR, inp.permP, GP, inp.dz64[rows])
+        rows_t = torch.from_numpy(rows).cuda()
+        check(host64(z[rows_t]), zo, "bf16", f"{name}[{layer}] z rows")
+        check(host64(dx[rows_t]), dxo, "bf16", f"{name}[{layer}] dx rows")
+        nR, nP = inp.m // inp.b, inp.n // inp.b
+        for side, nblk, q, dq in (("R", nR, inp.qR, dqR), ("P", nP, inp.qP, dqP)):
+            blocks = sorted({0, nblk // 2, nblk - 1})
+            dGs = oracle.grad_G_blocks(inp.x64, W0, inp.permR, GR, inp.permP, GP, inp.dz64, side, blocks)
+            dqo = np.stack([oracle.cnp_backward_block(q[j], inp.b, g) for j, g in zip(blocks, dGs)])
+            check(host64(dq)[blocks], dqo, "bf16", f"{name}[{layer}] dq{side} blocks {blocks}")
+        del L, z, dx, dqR, dqP
+        torch.cuda.empty_cache()
+
+
+def test_full_size_merge_down13b():
+    inp = pi.layer_inputs(pi.CONFIGS["down13b"], 0, T=256)
+    _merge_check(inp)

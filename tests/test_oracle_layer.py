@@ -116,18 +116,18 @@ def test_layer_gradients_match_central_differences():
                                    err_msg=name)
 
 
-def test_grad_G_block_matches_full_backward():
+def test_grad_G_blocks_match_full_backward():
     m, n, b, T = 24, 36, 6, 5
     X, W0, dZ, qR, qP, permR, permP = _case(m, n, b, T, 44)
     GR = oracle.cnp_blocks(qR, b)
     GP = oracle.cnp_blocks(qP, b)
     _, dGR, dGP = oracle.backward(X, W0, permR, GR, permP, GP, dZ)
+    got = oracle.grad_G_blocks(X, W0, permR, GR, permP, GP, dZ, "R", range(m // b))
     for j in range(m // b):
-        np.testing.assert_allclose(oracle.grad_G_block(X, W0, permR, GR, permP, GP, dZ, "R", j),
-                                   dGR[j], rtol=0, atol=1e-12 * np.abs(dGR).max())
-    for j in range(n // b):
-        np.testing.assert_allclose(oracle.grad_G_block(X, W0, permR, GR, permP, GP, dZ, "P", j),
-                                   dGP[j], rtol=0, atol=1e-12 * np.abs(dGP).max())
+        np.testing.assert_allclose(got[j], dGR[j], rtol=0, atol=1e-12 * np.abs(dGR).max())
+    got = oracle.grad_G_blocks(X, W0, permR, GR, permP, GP, dZ, "P", [5, 0, 3])
+    for g, j in zip(got, [5, 0, 3]):
+        np.testing.assert_allclose(g, dGP[j], rtol=0, atol=1e-12 * np.abs(dGP).max())
 
 
 def test_dq_linear_in_token_rows():
