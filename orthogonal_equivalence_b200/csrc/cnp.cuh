@@ -104,11 +104,26 @@ __global__ void identity_blocks_kernel(T* __restrict__ G, int nblk, int b) {
 
 __global__ void set_int_kernel(int32_t* p, int32_t v) { *p = v; }
 
-// fp32 copy of bf16 data (exact).
-__global__ void bf16_to_f32_kernel(const __nv_bfloat16* __restrict__ in, float* __restrict__ out, int64_t n) {
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
-    out[i] = __bfloat162float(in[i]);
+// out[t][c][r] = in[t][r][c] for b x b blocks (fp32 out; bf16 in is widened
+// exactly).  32 x 32 tiles through shared memory; grid (b/32, b/32, nblk),
+// block (32, 8).
+template <typename T>
+__global__ void transpose_blocks_kernel(const T* __restrict__ in, float* __restrict__ out, int b) {
+  __shared__ float tile[32][33];
+  const int64_t base = static_cast<int64_t>(blockIdx.z) * b * b;
+  const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int r = r0 + i, c = c0 + threadIdx.x;
+    if (r < b && c < b) {
+      if constexpr (std::is_same<T, float>::value) tile[i][threadIdx.x] = in[base + static_cast<int64_t>(r) * b + c];
+      else tile[i][threadIdx.x] = __bfloat162float(in[base + static_cast<int64_t>(r) * b + c]);
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int r = c0 + i, c = r0 + threadIdx.x;
+    if (r < b && c < b) out[base + static_cast<int64_t>(r) * b + c] = tile[threadIdx.x][i];
+  }
 }
 
 }  // namespace poetx

@@ -66,6 +66,9 @@ inline int choose_splits(int tiles, int K, int kblock, int sms, int min_kb = 4) 
 template <int BN, bool TF32>
 cudaError_t launch_tc_typed(const GemmDesc& g, cudaStream_t st, int device) {
   using C = tc::Cfg<BN, TF32>;
+  // tf32 operands are read as K-major tiles only (see nt_desc in poetx.cu).
+  if (TF32 && (g.A.mn_major || g.B.mn_major)) return cudaErrorNotSupported;
+  if (g.A.et != g.B.et) return cudaErrorInvalidValue;
   static bool attr_set[64] = {false};
   if (device >= 0 && device < 64 && !attr_set[device]) {
     cudaError_t e =

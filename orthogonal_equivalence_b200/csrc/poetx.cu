@@ -191,7 +191,7 @@ int dg_splits(int nblk, int b, int64_t T, int32_t dtype) {
 }
 
 size_t cnp_build_ws(int32_t nblk, int32_t b) { return 3 * al(sizeof(float) * size_t(nblk) * b * b); }
-size_t cnp_bwd_ws(int32_t nblk, int32_t b) { return 7 * al(sizeof(float) * size_t(nblk) * b * b); }
+size_t cnp_bwd_ws(int32_t nblk, int32_t b) { return 9 * al(sizeof(float) * size_t(nblk) * b * b); }
 
 size_t fwd_ws(const poetx_layer* L, int64_t T) {
   const size_t es = dtype_size(L->dtype);
@@ -376,23 +376,23 @@ GemmDesc blockgrad_desc(const void* in1, const void* in2, int et, int64_t T, int
   return g;
 }
 
-// Square b x b products over nblk blocks of fp32 scratch: C_t = opA(X_t) opB(Y_t).
-// opA: false -> X_t, true -> X_t^T.  opB: false -> Y_t, true -> Y_t^T.
-GemmDesc square_desc(const float* X, bool tA, const float* Y, bool tB, int nblk, int b, void* out, int et_out) {
+// Square b x b products over nblk blocks of fp32 scratch, in "NT" form:
+//   C_t = alpha * X_t Y_t^T   (both operands K-major)
+// Every tf32 product is written this way (tcgen05 tf32 reads K-major tiles of
+// the 128-byte swizzle; the MN-major fp32 tile layout is not used).
+GemmDesc nt_desc(const float* X, const float* Y, int nblk, int b, void* out, int et_out, float alpha = 1.f) {
   GemmDesc g;
   g.M = b;
   g.N = b;
   g.K = b;
   g.batch = nblk;
-  // A(i, k) = X[i][k]  -> K-major view (row = i + t b, col = k)
-  // A(i, k) = X[k][i]  -> MN-major view (row = k + t b, col = i)
-  g.A = blocks_view(X, ET_F32, nblk, b, !tA);
-  // B(k, n) = Y[k][n]  -> MN-major;  B(k, n) = Y[n][k] -> K-major
-  g.B = blocks_view(Y, ET_F32, nblk, b, tB);
+  g.A = blocks_view(X, ET_F32, nblk, b, true);  // A(i, k) = X[i][k]
+  g.B = blocks_view(Y, ET_F32, nblk, b, true);  // B(k, n) = Y[n][k]
   g.C.ptr = out;
   g.C.et = et_out;
   g.C.ld = b;
   g.C.batch_stride = int64_t(b) * b;
+  g.alpha = alpha;
   return g;
 }
 
@@ -406,6 +406,11 @@ AddDesc add_blocks(const float* p, int b, float beta) {
 }
 
 // ---------------------------------------------------------------- CNP
+// With Q skew (Q^T = -Q) and S = Q^2 symmetric, every product the
+// Cayley-Neumann block and its backward need is an X Y^T product:
+//   S   = Q Q    = -(Q Q^T)
+//   H S = H S^T                       (H = 2Q + S)
+//   G   = I + 2Q + 2S + H S           (= (I+Q)(I+Q+Q^2+Q^3))
 poetx_status cnp_build_impl(int32_t nblk, int32_t b, const float* q, int32_t dtype, void* G, Carver& ws,
                             cudaStream_t st, int device) {
   const size_t nbb = size_t(nblk) * b * b;
@@ -413,15 +418,13 @@ poetx_status cnp_build_impl(int32_t nblk, int32_t b, const float* q, int32_t dty
   float* S = ws.take<float>(sizeof(float) * nbb);
   float* H = ws.take<float>(sizeof(float) * nbb);
   const bool tc_path = use_tc(dtype);
-  PROFILED(ST_CNP_ELEM, st, unpack_skew_kernel<<<static_cast<int>((int64_t(nblk) * b + 7) / 8), 256, 0, st>>>(q, nblk, b, Q));
+  PROFILED(ST_CNP_ELEM, st,
+           unpack_skew_kernel<<<static_cast<int>((int64_t(nblk) * b + 7) / 8), 256, 0, st>>>(q, nblk, b, Q));
   POETX_CUDA(cudaGetLastError());
-  // S = Q Q
-  PROFILED(ST_CNP_GEMM, st, POETX_CUDA(launch_gemm(square_desc(Q, false, Q, false, nblk, b, S, ET_F32), tc_path, st, device)));
-  // H = 2Q + S
+  PROFILED(ST_CNP_GEMM, st, POETX_CUDA(launch_gemm(nt_desc(Q, Q, nblk, b, S, ET_F32, -1.f), tc_path, st, device)));
   PROFILED(ST_CNP_ELEM, st, axpby_kernel<<<grid_for(nbb, 256, device), 256, 0, st>>>(Q, 2.f, S, 1.f, H, nbb));
   POETX_CUDA(cudaGetLastError());
-  // G = H S + 2Q + 2S + I
-  GemmDesc g = square_desc(H, false, S, false, nblk, b, G, elem_type(dtype));
+  GemmDesc g = nt_desc(H, S, nblk, b, G, elem_type(dtype));
   g.add1 = add_blocks(Q, b, 2.f);
   g.add2 = add_blocks(S, b, 2.f);
   g.diag = 1.f;
@@ -432,45 +435,56 @@ poetx_status cnp_build_impl(int32_t nblk, int32_t b, const float* q, int32_t dty
 // dq from dG for G = I + 2A + 2S + H S with S = A A, H = 2A + S:
 //   dH = dG S^T;  dS = 2 dG + H^T dG + dH;  dA = 2 dG + 2 dH + dS A^T + A^T dS;
 //   dq_k = dA[i][j] - dA[j][i].
+// In X Y^T form: H^T dG = (H^T)(dG^T)^T, A^T dS = -(A)(dS^T)^T.
 poetx_status cnp_backward_impl(int32_t nblk, int32_t b, const float* q, const float* dG, float* dq,
                                int32_t accumulate, int32_t dtype, Carver& ws, cudaStream_t st, int device) {
   const size_t nbb = size_t(nblk) * b * b;
   float* A = ws.take<float>(sizeof(float) * nbb);
   float* S = ws.take<float>(sizeof(float) * nbb);
   float* H = ws.take<float>(sizeof(float) * nbb);
+  float* Ht = ws.take<float>(sizeof(float) * nbb);
+  float* dGt = ws.take<float>(sizeof(float) * nbb);
   float* dH = ws.take<float>(sizeof(float) * nbb);
   float* dS = ws.take<float>(sizeof(float) * nbb);
+  float* dSt = ws.take<float>(sizeof(float) * nbb);
   float* T1 = ws.take<float>(sizeof(float) * nbb);
-  float* dA = ws.take<float>(sizeof(float) * nbb);
+  float* dA = H;  // H is dead once Ht exists
   const bool tc_path = use_tc(dtype);
-  PROFILED(ST_CNP_ELEM, st, unpack_skew_kernel<<<static_cast<int>((int64_t(nblk) * b + 7) / 8), 256, 0, st>>>(q, nblk, b, A));
+  const dim3 tgrid((b + 31) / 32, (b + 31) / 32, nblk), tblock(32, 8);
+  PROFILED(ST_CNP_ELEM, st,
+           unpack_skew_kernel<<<static_cast<int>((int64_t(nblk) * b + 7) / 8), 256, 0, st>>>(q, nblk, b, A));
   POETX_CUDA(cudaGetLastError());
-  PROFILED(ST_CNP_GEMM, st, POETX_CUDA(launch_gemm(square_desc(A, false, A, false, nblk, b, S, ET_F32), tc_path, st, device)));
+  PROFILED(ST_CNP_GEMM, st, POETX_CUDA(launch_gemm(nt_desc(A, A, nblk, b, S, ET_F32, -1.f), tc_path, st, device)));
   PROFILED(ST_CNP_ELEM, st, axpby_kernel<<<grid_for(nbb, 256, device), 256, 0, st>>>(A, 2.f, S, 1.f, H, nbb));
+  PROFILED(ST_CNP_ELEM, st, transpose_blocks_kernel<<<tgrid, tblock, 0, st>>>(H, Ht, b));
+  PROFILED(ST_CNP_ELEM, st, transpose_blocks_kernel<<<tgrid, tblock, 0, st>>>(dG, dGt, b));
   POETX_CUDA(cudaGetLastError());
   // dH = dG S^T
-  PROFILED(ST_CNP_GEMM, st, POETX_CUDA(launch_gemm(square_desc(dG, false, S, true, nblk, b, dH, ET_F32), tc_path, st, device)));
+  PROFILED(ST_CNP_GEMM, st, POETX_CUDA(launch_gemm(nt_desc(dG, S, nblk, b, dH, ET_F32), tc_path, st, device)));
   // dS = H^T dG + 2 dG + dH
   {
-    GemmDesc g = square_desc(H, true, dG, false, nblk, b, dS, ET_F32);
+    GemmDesc g = nt_desc(Ht, dGt, nblk, b, dS, ET_F32);
     g.add1 = add_blocks(dG, b, 2.f);
     g.add2 = add_blocks(dH, b, 1.f);
     PROFILED(ST_CNP_GEMM, st, POETX_CUDA(launch_gemm(g, tc_path, st, device)));
   }
+  PROFILED(ST_CNP_ELEM, st, transpose_blocks_kernel<<<tgrid, tblock, 0, st>>>(dS, dSt, b));
+  POETX_CUDA(cudaGetLastError());
   // T1 = dS A^T + 2 dG + 2 dH
   {
-    GemmDesc g = square_desc(dS, false, A, true, nblk, b, T1, ET_F32);
+    GemmDesc g = nt_desc(dS, A, nblk, b, T1, ET_F32);
     g.add1 = add_blocks(dG, b, 2.f);
     g.add2 = add_blocks(dH, b, 2.f);
     PROFILED(ST_CNP_GEMM, st, POETX_CUDA(launch_gemm(g, tc_path, st, device)));
   }
-  // dA = A^T dS + T1
+  // dA = A^T dS + T1 = -(A dS^T^T) + T1
   {
-    GemmDesc g = square_desc(A, true, dS, false, nblk, b, dA, ET_F32);
+    GemmDesc g = nt_desc(A, dSt, nblk, b, dA, ET_F32, -1.f);
     g.add1 = add_blocks(T1, b, 1.f);
     PROFILED(ST_CNP_GEMM, st, POETX_CUDA(launch_gemm(g, tc_path, st, device)));
   }
-  PROFILED(ST_CNP_ELEM, st, fold_skew_kernel<<<static_cast<int>(int64_t(nblk) * b), 128, 0, st>>>(dA, nblk, b, dq, accumulate));
+  PROFILED(ST_CNP_ELEM, st,
+           fold_skew_kernel<<<static_cast<int>(int64_t(nblk) * b), 128, 0, st>>>(dA, nblk, b, dq, accumulate));
   POETX_CUDA(cudaGetLastError());
   return POETX_OK;
 }
@@ -758,9 +772,9 @@ poetx_status poetx_merge(const poetx_layer* layer, const int32_t* new_permR, con
   const int nR = L.m / L.b, nP = L.n / L.b;
   const size_t nm = size_t(L.n) * L.m;
   Carver c(ws, ws_bytes);
-  float* B1 = c.take<float>(sizeof(float) * nm);
+  float* B1t = c.take<float>(sizeof(float) * nm);
   float* At = c.take<float>(sizeof(float) * nm);
-  float* GPf = c.take<float>(sizeof(float) * size_t(nP) * L.b * L.b);
+  float* GPt = c.take<float>(sizeof(float) * size_t(nP) * L.b * L.b);
   int32_t* invR = c.take<int32_t>(sizeof(int32_t) * L.m);
   int32_t* invP = c.take<int32_t>(sizeof(int32_t) * L.n);
   int32_t* sigR = c.take<int32_t>(sizeof(int32_t) * L.m);
@@ -769,50 +783,38 @@ poetx_status poetx_merge(const poetx_layer* layer, const int32_t* new_permR, con
   // Stored W~ = (Psi_R W0 Psi_P^T)^T.  New weight R W0 P in the old frame is
   // A' = Diag(G_R) W~ Diag(G_P), stored transposed:
   //   At = Diag(G_P)^T . W . Diag(G_R)^T     ([n][m])
-  // pass 1: B1 = W . Diag(G_R)^T  (column blocks i: B1[:, ib:] = W[:, ib:] G_Ri^T)
+  // pass 1: B1t = Diag(G_R) . W^T ([m][n]); block i: B1t[ib + r][c] = sum_k G_Ri[r][k] W[c][ib + k]
   {
     GemmDesc g;
-    g.M = L.n;
-    g.N = L.b;
+    g.M = L.b;
+    g.N = L.n;
     g.K = L.b;
     g.batch = nR;
-    g.A = colblocks_view(L.W, et, L.n, L.m, L.b);
-    g.B = blocks_view(L.GR, et, nR, L.b, true);
-    g.C.ptr = B1;
+    g.A = blocks_view(L.GR, et, nR, L.b, true);          // A(r, k) = G_Ri[r][k]
+    g.B = colblocks_view(L.W, et, L.n, L.m, L.b);        // B(k, c) = W[c][ib + k]
+    g.C.ptr = B1t;
     g.C.et = ET_F32;
-    g.C.ld = L.m;
-    g.C.batch_stride = L.b;
+    g.C.ld = L.n;
+    g.C.batch_stride = int64_t(L.b) * L.n;
     PROFILED(ST_MERGE, st, POETX_CUDA(launch_gemm(g, tc_path, st, dev)));
   }
-  // pass 2: At[jb:(j+1)b, :] = G_Pj^T . B1[jb:(j+1)b, :]
+  // pass 2: At[jb + r][c] = sum_k G_Pj[k][r] B1t[c][jb + k]  (G_Pj^T, fp32, K-major)
   {
-    const float* GPsrc;
-    if (L.dtype == POETX_BF16) {
-      const int64_t cnt = int64_t(nP) * L.b * L.b;
-      bf16_to_f32_kernel<<<grid_for(cnt, 256, dev), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(L.GP), GPf, cnt);
-      POETX_CUDA(cudaGetLastError());
-      GPsrc = GPf;
-    } else {
-      GPsrc = static_cast<const float*>(L.GP);
-    }
+    const dim3 tgrid((L.b + 31) / 32, (L.b + 31) / 32, nP), tblock(32, 8);
+    if (L.dtype == POETX_BF16)
+      PROFILED(ST_MERGE, st, transpose_blocks_kernel<<<tgrid, tblock, 0, st>>>(
+                                 static_cast<const __nv_bfloat16*>(L.GP), GPt, L.b));
+    else
+      PROFILED(ST_MERGE, st,
+               transpose_blocks_kernel<<<tgrid, tblock, 0, st>>>(static_cast<const float*>(L.GP), GPt, L.b));
+    POETX_CUDA(cudaGetLastError());
     GemmDesc g;
     g.M = L.b;
     g.N = L.m;
     g.K = L.b;
     g.batch = nP;
-    // A(r, k) = G_Pj[k][r]: MN-major view of the blocks
-    g.A = blocks_view(GPsrc, ET_F32, nP, L.b, false);
-    // B(k, c) = B1[jb + k][c]: MN-major view, batch moves down b rows
-    Operand2D b;
-    b.ptr = B1;
-    b.et = ET_F32;
-    b.rows = L.n;
-    b.cols = L.m;
-    b.ld = L.m;
-    b.mn_major = true;
-    b.b_row = L.b;
-    b.b_col = 0;
-    g.B = b;
+    g.A = blocks_view(GPt, ET_F32, nP, L.b, true);       // A(r, k) = G_Pj[k][r]
+    g.B = colblocks_view(B1t, ET_F32, L.m, L.n, L.b);    // B(k, c) = B1t[c][jb + k]
     g.C.ptr = At;
     g.C.et = ET_F32;
     g.C.ld = L.m;
