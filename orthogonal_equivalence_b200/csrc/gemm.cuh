@@ -126,50 +126,82 @@ struct Params {
   EpiParams epi;
 };
 
-template <int BN, bool TF32>
+// Two operand-feeding modes:
+//  * streamed  (B_RES = false): every pipeline stage carries one K-block of A
+//    and of B; tiles are dealt to the persistent CTAs round-robin, M-tiles
+//    grouped GROUP_M at a time so a B panel is reused from L2;
+//  * B-resident (B_RES = true): the whole K-range of the B tile (a b x b block
+//    of Diag(G) for the block-diagonal products) is loaded once into shared
+//    memory and kept while the CTA streams a contiguous run of M-tiles (token
+//    tiles) of A through the stages; B is reloaded only when the block changes.
+template <int BN, bool TF32, bool B_RES>
 struct Cfg {
   static constexpr int ESZ = TF32 ? 4 : 2;
   static constexpr int CH = 128 / ESZ;  // elements per 128-byte swizzle row = K per stage
   static constexpr int UMMA_K = TF32 ? 8 : 16;
   static constexpr int A_BYTES = BM * 128;
   static constexpr int B_BYTES = BN * 128;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
+  static constexpr int STAGE_BYTES = B_RES ? A_BYTES : A_BYTES + B_BYTES;
+  static constexpr int STAGES = B_RES ? 5 : (BN == 256 ? 4 : (BN == 128 ? 6 : 8));
+  static constexpr int MAX_KB_RES = B_RES ? (128 * 1024) / B_BYTES : 0;  // resident K-blocks of B
   static constexpr int TMEM_COLS = 2 * BN;  // double-buffered fp32 accumulator
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + MAX_KB_RES * B_BYTES + 1024 + 256;
 };
 
+// Streamed mode: round-robin tiles, GROUP_M-grouped raster inside each
+// (batch, split).  B-resident mode: contiguous tiles, M fastest.
+template <bool B_RES>
 __device__ __forceinline__ void decode_tile(const Params& p, int tile, int& bt, int& sp, int& mt, int& nt) {
   const int per = p.tiles_m * p.tiles_n;
   const int bs = tile / per;
   int r = tile - bs * per;
   bt = bs / p.splits;
   sp = bs - bt * p.splits;
-  const int group_span = GROUP_M * p.tiles_n;
-  const int g = r / group_span;
-  const int first_m = g * GROUP_M;
-  const int gsize = min(p.tiles_m - first_m, GROUP_M);
-  r -= g * group_span;
-  mt = first_m + r % gsize;
-  nt = r / gsize;
+  if constexpr (B_RES) {
+    nt = r / p.tiles_m;
+    mt = r - nt * p.tiles_m;
+  } else {
+    const int group_span = GROUP_M * p.tiles_n;
+    const int g = r / group_span;
+    const int first_m = g * GROUP_M;
+    const int gsize = min(p.tiles_m - first_m, GROUP_M);
+    r -= g * group_span;
+    mt = first_m + r % gsize;
+    nt = r / gsize;
+  }
 }
 
-template <int BN, bool TF32>
+// Tiles of this CTA: [t0, t1) with stride `step`.
+template <bool B_RES>
+__device__ __forceinline__ void tile_range(int total, int& t0, int& t1, int& step) {
+  if constexpr (B_RES) {
+    t0 = static_cast<int>(static_cast<int64_t>(blockIdx.x) * total / gridDim.x);
+    t1 = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * total / gridDim.x);
+    step = 1;
+  } else {
+    t0 = blockIdx.x;
+    t1 = total;
+    step = gridDim.x;
+  }
+}
+
+template <int BN, bool TF32, bool B_RES>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, Params p) {
-  using C = Cfg<BN, TF32>;
+  using C = Cfg<BN, TF32, B_RES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
-  // bars: full[STAGES], empty[STAGES], tfull[2], tempty[2], drain
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * C::STAGES + 5);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES + C::MAX_KB_RES * C::B_BYTES);
+  // bars: full[STAGES], empty[STAGES], tfull[2], tempty[2], drain, bfull, bempty
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * C::STAGES + 7);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t smem_base = smem_u32(smem);
+  const uint32_t sB_res = smem_base + C::STAGES * C::STAGE_BYTES;  // resident B (B_RES only)
   auto bar = [&](int i) { return smem_u32(bars + i); };
   const int FULL = 0, EMPTY = C::STAGES, TFULL = 2 * C::STAGES, TEMPTY = 2 * C::STAGES + 2,
-            DRAIN = 2 * C::STAGES + 4;
+            DRAIN = 2 * C::STAGES + 4, BFULL = 2 * C::STAGES + 5, BEMPTY = 2 * C::STAGES + 6;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -181,6 +213,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(bar(TEMPTY + a), 128);
     }
     mbar_init(bar(DRAIN), 1);
+    mbar_init(bar(BFULL), 1);
+    mbar_init(bar(BEMPTY), 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -193,6 +227,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem_base = *tmem_holder;
 
   const int total = p.batch * p.splits * p.tiles_m * p.tiles_n;
+  int t0, t1, tstep;
+  tile_range<B_RES>(total, t0, t1, tstep);
+  // key of the resident B tile: (batch, split, n-tile)
+  auto b_key = [&](int bt, int sp, int nt) { return (bt * p.splits + sp) * p.tiles_n + nt; };
 
   if (warp == 0) {
     if (lane == 0) {
@@ -202,14 +240,40 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       uint32_t armed = 0, armed_phase = 0;  // per-stage bits for the abort drain
+      int key_prev = -1;
+      uint32_t bloads = 0;
+      bool b_armed = false;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      for (int tile = t0; tile < t1 && ok; tile += tstep) {
         int bt, sp, mt, nt;
-        decode_tile(p, tile, bt, sp, mt, nt);
+        decode_tile<B_RES>(p, tile, bt, sp, mt, nt);
         const int kbeg = sp * p.k_per_split;
         const int kend = min(p.K, kbeg + p.k_per_split);
         const int nkb = (kend - kbeg + C::CH - 1) / C::CH;
         const int m0 = mt * BM, n0 = nt * BN;
+        if constexpr (B_RES) {
+          const int key = b_key(bt, sp, nt);
+          if (key != key_prev) {
+            // the previous resident B is free once the MMAs that read it are done
+            if (bloads > 0 && !mbar_wait(bar(BEMPTY), (bloads - 1) & 1u, DERR_GEMM_WAIT)) { ok = false; break; }
+            const uint32_t fb = bar(BFULL);
+            mbar_arrive_expect_tx(fb, nkb * C::B_BYTES);
+            b_armed = true;
+            for (int kb = 0; kb < nkb; ++kb) {
+              const int k = kbeg + kb * C::CH;
+              const uint32_t sb = sB_res + kb * C::B_BYTES;
+              if (!p.b_mn) {
+                tma_load_2d(sb, &tmB, fb, k + bt * p.b_bcol, n0 + bt * p.b_brow);
+              } else {
+#pragma unroll
+                for (int c = 0; c < BN / C::CH; ++c)
+                  tma_load_2d(sb + c * (C::CH * 128), &tmB, fb, n0 + c * C::CH + bt * p.b_bcol, k + bt * p.b_brow);
+              }
+            }
+            ++bloads;
+            key_prev = key;
+          }
+        }
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(bar(EMPTY + stage), phase ^ 1u, DERR_GEMM_WAIT)) { ok = false; break; }
           const uint32_t fb = bar(FULL + stage);
@@ -217,7 +281,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           armed |= 1u << stage;
           armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
           const uint32_t sa = smem_base + stage * C::STAGE_BYTES;
-          const uint32_t sb = sa + C::A_BYTES;
           const int k = kbeg + kb * C::CH;
           if (!p.a_mn) {
             tma_load_2d(sa, &tmA, fb, k + bt * p.a_bcol, m0 + bt * p.a_brow);
@@ -226,12 +289,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int c = 0; c < BM / C::CH; ++c)
               tma_load_2d(sa + c * (C::CH * 128), &tmA, fb, m0 + c * C::CH + bt * p.a_bcol, k + bt * p.a_brow);
           }
-          if (!p.b_mn) {
-            tma_load_2d(sb, &tmB, fb, k + bt * p.b_bcol, n0 + bt * p.b_brow);
-          } else {
+          if constexpr (!B_RES) {
+            const uint32_t sb = sa + C::A_BYTES;
+            if (!p.b_mn) {
+              tma_load_2d(sb, &tmB, fb, k + bt * p.b_bcol, n0 + bt * p.b_brow);
+            } else {
 #pragma unroll
-            for (int c = 0; c < BN / C::CH; ++c)
-              tma_load_2d(sb + c * (C::CH * 128), &tmB, fb, n0 + c * C::CH + bt * p.b_bcol, k + bt * p.b_brow);
+              for (int c = 0; c < BN / C::CH; ++c)
+                tma_load_2d(sb + c * (C::CH * 128), &tmB, fb, n0 + c * C::CH + bt * p.b_bcol, k + bt * p.b_brow);
+            }
           }
           if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -240,22 +306,40 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // Let the copies already issued land before the block exits.
         for (int s = 0; s < C::STAGES; ++s)
           if (armed & (1u << s)) mbar_wait(bar(FULL + s), (armed_phase >> s) & 1u, DERR_GEMM_WAIT);
+        if (b_armed) mbar_wait(bar(BFULL), (bloads - 1) & 1u, DERR_GEMM_WAIT);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- MMA issuer
-      const uint32_t a_base_lbo = p.a_lbo, b_base_lbo = p.b_lbo;
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
+      int key_prev = -1;
+      uint32_t bwaits = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++local) {
+      for (int tile = t0; tile < t1 && ok; tile += tstep, ++local) {
         int bt, sp, mt, nt;
-        decode_tile(p, tile, bt, sp, mt, nt);
+        decode_tile<B_RES>(p, tile, bt, sp, mt, nt);
         const int kbeg = sp * p.k_per_split;
         const int kend = min(p.K, kbeg + p.k_per_split);
         const int nkb = (kend - kbeg + C::CH - 1) / C::CH;
+        bool last_of_key = false;
+        if constexpr (B_RES) {
+          const int key = b_key(bt, sp, nt);
+          if (key != key_prev) {
+            if (!mbar_wait(bar(BFULL), bwaits & 1u, DERR_GEMM_WAIT)) { ok = false; break; }
+            ++bwaits;
+            key_prev = key;
+          }
+          if (tile + tstep >= t1) {
+            last_of_key = true;
+          } else {
+            int bt2, sp2, mt2, nt2;
+            decode_tile<B_RES>(p, tile + tstep, bt2, sp2, mt2, nt2);
+            last_of_key = b_key(bt2, sp2, nt2) != key;
+          }
+        }
         const int acc = local & 1;
         const uint32_t acc_phase = (local >> 1) & 1;
         if (!mbar_wait(bar(TEMPTY + acc), acc_phase ^ 1u, DERR_GEMM_WAIT)) { ok = false; break; }
@@ -265,11 +349,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (!mbar_wait(bar(FULL + stage), phase, DERR_GEMM_WAIT)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_base + stage * C::STAGE_BYTES;
-          const uint32_t sb = sa + C::A_BYTES;
+          const uint32_t sb = B_RES ? sB_res + kb * C::B_BYTES : sa + C::A_BYTES;
 #pragma unroll
           for (int kk = 0; kk < C::CH / C::UMMA_K; ++kk) {
-            const uint64_t da = smem_desc_sw128(sa + kk * p.a_kstep, a_base_lbo, 1024);
-            const uint64_t db = smem_desc_sw128(sb + kk * p.b_kstep, b_base_lbo, 1024);
+            const uint64_t da = smem_desc_sw128(sa + kk * p.a_kstep, p.a_lbo, 1024);
+            const uint64_t db = smem_desc_sw128(sb + kk * p.b_kstep, p.b_lbo, 1024);
             tc_mma<TF32>(d_tmem, da, db, p.idesc, (kb | kk) != 0 ? 1u : 0u);
           }
           tc_commit(bar(EMPTY + stage));
@@ -277,6 +361,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         if (!ok) break;
         tc_commit(bar(TFULL + acc));
+        if (B_RES && last_of_key) tc_commit(bar(BEMPTY));
       }
       // All MMAs issued by this thread have completed once DRAIN fires.
       tc_commit(bar(DRAIN));
@@ -287,9 +372,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter + 32)
     const EpiParams& e = p.epi;
     int local = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
+    for (int tile = t0; tile < t1; tile += tstep, ++local) {
       int bt, sp, mt, nt;
-      decode_tile(p, tile, bt, sp, mt, nt);
+      decode_tile<B_RES>(p, tile, bt, sp, mt, nt);
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
       bool ok = mbar_wait(bar(TFULL + acc), acc_phase, DERR_GEMM_WAIT);
@@ -306,8 +391,37 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int64_t n0 = static_cast<int64_t>(nt) * BN + c0;
         if (!row_ok) continue;
         if (n0 + 32 <= e.N) {
+          // alpha * acc + beta1 X1 + beta2 X2 + diag I; the addends are read
+          // as 16-byte vectors (host guarantees 16-byte alignment)
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = epi_value(e, v[i], bt, r, n0 + i);
+          for (int i = 0; i < 32; ++i) v[i] *= e.alpha;
+          if (e.x1) {
+            const float4* xp = reinterpret_cast<const float4*>(e.x1 + bt * e.x1_bs + r * e.x1_ld + n0);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const float4 a = __ldg(xp + q);
+              v[4 * q] += e.beta1 * a.x;
+              v[4 * q + 1] += e.beta1 * a.y;
+              v[4 * q + 2] += e.beta1 * a.z;
+              v[4 * q + 3] += e.beta1 * a.w;
+            }
+          }
+          if (e.x2) {
+            const float4* xp = reinterpret_cast<const float4*>(e.x2 + bt * e.x2_bs + r * e.x2_ld + n0);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const float4 a = __ldg(xp + q);
+              v[4 * q] += e.beta2 * a.x;
+              v[4 * q + 1] += e.beta2 * a.y;
+              v[4 * q + 2] += e.beta2 * a.z;
+              v[4 * q + 3] += e.beta2 * a.w;
+            }
+          }
+          if (e.diag != 0.f && r >= n0 && r < n0 + 32) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (r == n0 + i) v[i] += e.diag;
+          }
           if (e.c_et == ET_BF16) {
             uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(e.c) + obase + n0);
 #pragma unroll

@@ -53,26 +53,27 @@ inline bool encode_map(CUtensorMap* map, const Operand2D& op, int box_outer) {
   return r == CUDA_SUCCESS;
 }
 
-// Split-K count so that (tiles x splits) fills about `waves` of the SMs while
-// every split keeps at least `min_kb` K-blocks.
-inline int choose_splits(int tiles, int K, int kblock, int sms, int min_kb = 4) {
-  const int nkb = (K + kblock - 1) / kblock;
-  int s = 1;
-  while (tiles * s * 2 <= sms * 2 && nkb / (s * 2) >= min_kb) s *= 2;
-  while (tiles * s < sms && nkb / (s + 1) >= min_kb) ++s;
-  return s;
-}
-
-template <int BN, bool TF32>
+template <int BN, bool TF32, bool B_RES>
 cudaError_t launch_tc_typed(const GemmDesc& g, cudaStream_t st, int device) {
-  using C = tc::Cfg<BN, TF32>;
+  using C = tc::Cfg<BN, TF32, B_RES>;
   // tf32 operands are read as K-major tiles only (see nt_desc in poetx.cu).
   if (TF32 && (g.A.mn_major || g.B.mn_major)) return cudaErrorNotSupported;
   if (g.A.et != g.B.et) return cudaErrorInvalidValue;
+  // the epilogue reads addends and writes full 32-column chunks as 16-byte vectors
+  auto vec_ok = [](const AddDesc& a) {
+    return !a.ptr || ((reinterpret_cast<uintptr_t>(a.ptr) & 15u) == 0 && a.ld % 4 == 0 && a.batch_stride % 4 == 0);
+  };
+  if (!vec_ok(g.add1) || !vec_ok(g.add2)) return cudaErrorInvalidValue;
+  {
+    const int v = g.C.et == ET_BF16 ? 8 : 4;
+    if ((reinterpret_cast<uintptr_t>(g.C.ptr) & 15u) != 0 || g.C.ld % v != 0 || g.C.batch_stride % v != 0 ||
+        g.C.split_stride % v != 0)
+      return cudaErrorInvalidValue;
+  }
   static bool attr_set[64] = {false};
   if (device >= 0 && device < 64 && !attr_set[device]) {
     cudaError_t e =
-        cudaFuncSetAttribute(tc::gemm_kernel<BN, TF32>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+        cudaFuncSetAttribute(tc::gemm_kernel<BN, TF32, B_RES>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set[device] = true;
   }
@@ -111,7 +112,8 @@ cudaError_t launch_tc_typed(const GemmDesc& g, cudaStream_t st, int device) {
   const int total = g.batch * g.splits * p.tiles_m * p.tiles_n;
   const int grid = total < sm_count(device) ? total : sm_count(device);
   if (grid <= 0) return cudaSuccess;
-  tc::gemm_kernel<BN, TF32><<<grid, tc::NUM_THREADS, C::SMEM_BYTES, st>>>(ma, mb, p);
+  if (B_RES && p.k_per_split > C::MAX_KB_RES * C::CH) return cudaErrorInvalidValue;
+  tc::gemm_kernel<BN, TF32, B_RES><<<grid, tc::NUM_THREADS, C::SMEM_BYTES, st>>>(ma, mb, p);
   return cudaGetLastError();
 }
 
@@ -123,12 +125,23 @@ inline int choose_bn(int N) {
   return 64;
 }
 
+// B stays resident when its whole K-range fits the resident area and enough
+// M-tiles share it (block-diagonal products: K = N = b, M = tokens).
+template <int BN, bool TF32>
+cudaError_t launch_tc_bn(const GemmDesc& g, cudaStream_t st, int device) {
+  using CR = tc::Cfg<BN, TF32, true>;
+  const int tiles_m = (g.M + tc::BM - 1) / tc::BM;
+  const int nkb = (g.K + CR::CH - 1) / CR::CH;
+  const bool resident = g.splits == 1 && nkb <= CR::MAX_KB_RES && tiles_m >= 4;
+  return resident ? launch_tc_typed<BN, TF32, true>(g, st, device) : launch_tc_typed<BN, TF32, false>(g, st, device);
+}
+
 inline cudaError_t launch_tc(const GemmDesc& g, cudaStream_t st, int device) {
   const bool tf32 = g.A.et == ET_F32;
   switch (choose_bn(g.N)) {
-    case 256: return tf32 ? launch_tc_typed<256, true>(g, st, device) : launch_tc_typed<256, false>(g, st, device);
-    case 128: return tf32 ? launch_tc_typed<128, true>(g, st, device) : launch_tc_typed<128, false>(g, st, device);
-    default: return tf32 ? launch_tc_typed<64, true>(g, st, device) : launch_tc_typed<64, false>(g, st, device);
+    case 256: return tf32 ? launch_tc_bn<256, true>(g, st, device) : launch_tc_bn<256, false>(g, st, device);
+    case 128: return tf32 ? launch_tc_bn<128, true>(g, st, device) : launch_tc_bn<128, false>(g, st, device);
+    default: return tf32 ? launch_tc_bn<64, true>(g, st, device) : launch_tc_bn<64, false>(g, st, device);
   }
 }
 

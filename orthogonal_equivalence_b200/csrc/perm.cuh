@@ -174,6 +174,112 @@ __global__ void __launch_bounds__(256) scatter_kernel(const T* __restrict__ in, 
   }
 }
 
+// Column permutation of row-major activations on the hot path, fed by bulk
+// copies.  out[r][c] = in[r][map[c]] (gather), or with `inverse` set
+// out[r][map[c]] = in[r][c] (scatter, done as a gather through the inverse
+// map, which every block first builds in shared memory).  Rows are contiguous
+// (leading dimension == cols), so a chunk of rows_per_stage rows is one
+// contiguous bulk copy; two stages are double-buffered: while the block
+// permutes one chunk out of shared memory, the next one is in flight.  Each
+// thread writes whole 16-byte vectors, so the global stores are coalesced.
+// Shared memory: cols 16-bit indices + 2 * rows_per_stage * cols * sizeof(T).
+template <typename T>
+__global__ void __launch_bounds__(256) permute_rows_kernel(const T* __restrict__ in, T* __restrict__ out, int64_t rows,
+                                                           int cols, const int32_t* __restrict__ map, int inverse,
+                                                           int rows_per_stage) {
+  extern __shared__ __align__(128) uint8_t sm_raw[];
+  __shared__ __align__(8) uint64_t full_bar[2];
+  constexpr int V = 16 / sizeof(T);
+  uint16_t* idx = reinterpret_cast<uint16_t*>(sm_raw);
+  const size_t idx_bytes = (static_cast<size_t>(cols) * 2 + 127) & ~size_t(127);
+  T* stage_base = reinterpret_cast<T*>(sm_raw + idx_bytes);
+  const int64_t stage_elems = static_cast<int64_t>(rows_per_stage) * cols;
+  const int64_t nchunks = (rows + rows_per_stage - 1) / rows_per_stage;
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&full_bar[0]), 1);
+    mbar_init(smem_u32(&full_bar[1]), 1);
+    fence_barrier_init();
+  }
+  if (inverse) {
+    // entries a non-bijective map never reaches stay 0 (in range)
+    for (int c = threadIdx.x; c < cols; c += blockDim.x) idx[c] = 0;
+    __syncthreads();
+  }
+  for (int c = threadIdx.x; c < cols; c += blockDim.x) {
+    const int m = map[c];
+    if (m < 0 || m >= cols) {
+      record_error(DERR_BAD_INDEX);
+      if (!inverse) idx[c] = 0;
+      continue;
+    }
+    if (inverse) idx[m] = static_cast<uint16_t>(c);
+    else idx[c] = static_cast<uint16_t>(m);
+  }
+  __syncthreads();
+
+  uint32_t pending = 0;  // stages with a copy in flight (thread 0's view)
+  auto issue = [&](int64_t chunk, int s) {
+    const int64_t r0 = chunk * rows_per_stage;
+    const int64_t nr = rows - r0 < rows_per_stage ? rows - r0 : rows_per_stage;
+    const uint32_t bytes = static_cast<uint32_t>(nr * cols * sizeof(T));
+    const uint32_t bar = smem_u32(&full_bar[s]);
+    // earlier generic-proxy reads of this stage (ordered by the block barrier)
+    // come before the async-proxy write
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    mbar_arrive_expect_tx(bar, bytes);
+    bulk_load(smem_u32(stage_base + s * stage_elems), in + r0 * cols, bytes, bar);
+    pending |= 1u << s;
+  };
+
+  int64_t chunk = blockIdx.x;
+  if (threadIdx.x == 0 && chunk < nchunks) issue(chunk, 0);
+  uint32_t phase[2] = {0u, 0u};
+  bool ok = true;
+  for (int it = 0; chunk < nchunks; chunk += gridDim.x, ++it) {
+    const int s = it & 1;
+    const int64_t next = chunk + gridDim.x;
+    if (threadIdx.x == 0 && next < nchunks) issue(next, s ^ 1);
+    ok = mbar_wait(smem_u32(&full_bar[s]), phase[s], DERR_PERM_WAIT);
+    if (ok) {
+      phase[s] ^= 1u;
+      pending &= ~(1u << s);
+    }
+    if (!__syncthreads_and(ok)) break;
+    const int64_t r0 = chunk * rows_per_stage;
+    const int nr = static_cast<int>(rows - r0 < rows_per_stage ? rows - r0 : rows_per_stage);
+    const T* st = stage_base + s * stage_elems;
+    const int vpr = cols / V;  // vectors per row
+    for (int v = threadIdx.x; v < nr * vpr; v += blockDim.x) {
+      const int rr = v / vpr;
+      const int c0 = (v - rr * vpr) * V;
+      const T* srow = st + static_cast<int64_t>(rr) * cols;
+      union {
+        uint4 u;
+        T e[V];
+      } pk;
+      if constexpr (V == 8) {
+        const uint4 ii = *reinterpret_cast<const uint4*>(idx + c0);
+        const uint16_t* iv = reinterpret_cast<const uint16_t*>(&ii);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) pk.e[k] = srow[iv[k]];
+      } else {
+        const uint2 ii = *reinterpret_cast<const uint2*>(idx + c0);
+        const uint16_t* iv = reinterpret_cast<const uint16_t*>(&ii);
+#pragma unroll
+        for (int k = 0; k < V; ++k) pk.e[k] = srow[iv[k]];
+      }
+      reinterpret_cast<uint4*>(out + (r0 + rr) * cols + c0)[0] = pk.u;
+    }
+    __syncthreads();  // stage s may be refilled next iteration
+  }
+  if (!ok && threadIdx.x == 0) {
+    // let a copy still in flight land before the block exits
+    for (int s = 0; s < 2; ++s)
+      if (pending & (1u << s)) mbar_wait(smem_u32(&full_bar[s]), phase[s], DERR_PERM_WAIT);
+  }
+}
+
 // inv[perm[i]] = i
 __global__ void invert_perm_kernel(const int32_t* __restrict__ perm, int32_t* __restrict__ inv, int len) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;

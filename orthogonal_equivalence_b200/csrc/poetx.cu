@@ -276,6 +276,44 @@ cudaError_t scatter(const T* in, int64_t ld_in, T* out, int64_t ld_out, int64_t 
   return cudaGetLastError();
 }
 
+// Hot-path column permutation of contiguous [rows][cols] activations:
+// out = in[:, map] (inverse == 0) or out[:, map] = in (inverse == 1).
+template <typename T>
+cudaError_t permute_cols(const T* in, T* out, int64_t rows, int cols, const int32_t* map, int inverse,
+                         cudaStream_t st, int device) {
+  if (rows <= 0 || cols <= 0) return cudaSuccess;
+  constexpr int V = 16 / sizeof(T);
+  const bool fast = cols < 65536 && cols % V == 0 && aligned16(in) && aligned16(out);
+  if (!fast) {
+    return inverse ? scatter(in, cols, out, cols, rows, rows, cols, map, nullptr, st, device)
+                   : gather(in, cols, rows, out, cols, rows, cols, map, nullptr, st, device);
+  }
+  static bool attr[64] = {false};
+  const size_t row_bytes = size_t(cols) * sizeof(T);
+  int rps = static_cast<int>((24 * 1024) / row_bytes);
+  if (rps < 1) rps = 1;
+  if (rps > 64) rps = 64;
+  const size_t idx_bytes = (size_t(cols) * 2 + 127) & ~size_t(127);
+  const size_t smem = idx_bytes + 2 * size_t(rps) * row_bytes;
+  if (smem > 200 * 1024) return cudaErrorInvalidValue;
+  cudaError_t e = allow_smem(permute_rows_kernel<T>, smem, &attr[device & 63]);
+  if (e != cudaSuccess) return e;
+  const int per_sm = static_cast<int>((220 * 1024) / (smem + 1024));
+  const int64_t chunks = (rows + rps - 1) / rps;
+  int64_t g = int64_t(sm_count(device)) * (per_sm < 1 ? 1 : (per_sm > 8 ? 8 : per_sm));
+  if (g > chunks) g = chunks;
+  permute_rows_kernel<T><<<static_cast<int>(g), 256, smem, st>>>(in, out, rows, cols, map, inverse, rps);
+  return cudaGetLastError();
+}
+
+cudaError_t permute_dt(int32_t dt, const void* in, void* out, int64_t rows, int cols, const int32_t* map, int inverse,
+                       cudaStream_t st, int device) {
+  if (dt == POETX_BF16)
+    return permute_cols(static_cast<const __nv_bfloat16*>(in), static_cast<__nv_bfloat16*>(out), rows, cols, map,
+                        inverse, st, device);
+  return permute_cols(static_cast<const float*>(in), static_cast<float*>(out), rows, cols, map, inverse, st, device);
+}
+
 cudaError_t gather_dt(int32_t dt, const void* in, int64_t ld_in, int64_t in_rows, void* out, int64_t ld_out,
                       int64_t rows, int cols, const int32_t* colmap, const int32_t* rowmap, cudaStream_t st,
                       int device) {
@@ -625,7 +663,7 @@ poetx_status poetx_forward(const poetx_layer* layer, int64_t T, const void* x, v
   void* Yw = c.take<uint8_t>(es * T * L.n);
   void* Y = y_save ? y_save : Yw;
   // Xg = x Psi_R^T  (columns gathered into the Psi_R frame)
-  PROFILED(ST_PERMUTE, st, POETX_CUDA(gather_dt(L.dtype, x, L.m, T, Xg, L.m, T, L.m, L.permR, nullptr, st, dev)));
+  PROFILED(ST_PERMUTE, st, POETX_CUDA(permute_dt(L.dtype, x, Xg, T, L.m, L.permR, 0, st, dev)));
   // U_j = Xg_j G_Rj
   PROFILED(ST_BLOCKDIAG, st, POETX_CUDA(launch_gemm(blockdiag_desc(Xg, et, T, L.m, L.b, L.GR, false, U, et), tc_path, st, dev)));
   // Y = U W~  (W~ = Psi_R W0 Psi_P^T stored [n][m]: B(k=i', n=j') = W[j'][i'], K-major)
@@ -651,7 +689,7 @@ poetx_status poetx_forward(const poetx_layer* layer, int64_t T, const void* x, v
   // V_j = Y_j G_Pj
   PROFILED(ST_BLOCKDIAG, st, POETX_CUDA(launch_gemm(blockdiag_desc(Y, et, T, L.n, L.b, L.GP, false, V, et), tc_path, st, dev)));
   // z = V Psi_P  (columns scattered back to natural order)
-  PROFILED(ST_PERMUTE, st, POETX_CUDA(scatter_dt(L.dtype, V, L.n, z, L.n, T, T, L.n, L.permP, nullptr, st, dev)));
+  PROFILED(ST_PERMUTE, st, POETX_CUDA(permute_dt(L.dtype, V, z, T, L.n, L.permP, 1, st, dev)));
   return POETX_OK;
 }
 
@@ -696,7 +734,7 @@ poetx_status poetx_backward(const poetx_layer* layer, int64_t T, const void* x, 
 
   // dV = dz Psi_P^T
   void* dV = bufA;
-  PROFILED(ST_PERMUTE, st, POETX_CUDA(gather_dt(L.dtype, dz, L.n, T, dV, L.n, T, L.n, L.permP, nullptr, st, dev)));
+  PROFILED(ST_PERMUTE, st, POETX_CUDA(permute_dt(L.dtype, dz, dV, T, L.n, L.permP, 0, st, dev)));
   // dY_j = dV_j G_Pj^T
   void* dY = bufB;
   PROFILED(ST_BLOCKDIAG, st, POETX_CUDA(launch_gemm(blockdiag_desc(dV, et, T, L.n, L.b, L.GP, true, dY, et), tc_path, st, dev)));
@@ -724,14 +762,14 @@ poetx_status poetx_backward(const poetx_layer* layer, int64_t T, const void* x, 
   }
   // Xg = x Psi_R^T (re-gathered; dV is dead)
   void* Xg = bufA;
-  PROFILED(ST_PERMUTE, st, POETX_CUDA(gather_dt(L.dtype, x, L.m, T, Xg, L.m, T, L.m, L.permR, nullptr, st, dev)));
+  PROFILED(ST_PERMUTE, st, POETX_CUDA(permute_dt(L.dtype, x, Xg, T, L.m, L.permR, 0, st, dev)));
   // dXg_j = dU_j G_Rj^T (dY is dead)
   void* dXg = bufB;
   if (dx) PROFILED(ST_BLOCKDIAG, st, POETX_CUDA(launch_gemm(blockdiag_desc(dU, et, T, L.m, L.b, L.GR, true, dXg, et), tc_path, st, dev)));
   // dG_Rj = Xg_j^T dU_j
   PROFILED(ST_DG, st, POETX_CUDA(launch_gemm(blockgrad_desc(Xg, dU, et, T, L.m, L.b, sR, partR), tc_path, st, dev)));
   // dx = dXg Psi_R
-  if (dx) PROFILED(ST_PERMUTE, st, POETX_CUDA(scatter_dt(L.dtype, dXg, L.m, dx, L.m, T, T, L.m, L.permR, nullptr, st, dev)));
+  if (dx) PROFILED(ST_PERMUTE, st, POETX_CUDA(permute_dt(L.dtype, dXg, dx, T, L.m, L.permR, 1, st, dev)));
   // dq from dG (fixed-order reduction of the token splits, then the CNP backward)
   PROFILED(ST_REDUCE, st,
            reduce_splits_kernel<<<grid_for(nP * bb / 4 + 1, 256, dev), 256, 0, st>>>(partP, sP, int64_t(nP) * bb, dG));

@@ -41,6 +41,8 @@ SMALL = [
     ("down13b", 1536, 1024, 512, 130),
     ("block8b", 1024, 256, 256, 257),
     ("block8b", 256, 768, 256, 1),
+    ("block8b", 512, 1024, 256, 1000),   # >= 4 token tiles: block-resident G path
+    ("down13b", 1024, 1536, 512, 777),
 ]
 
 
