@@ -109,6 +109,12 @@ poetx_status poetx_frame_export(const poetx_layer* layer, void* W0lin, void* str
 poetx_status poetx_cnp_build(int32_t nblk, int32_t b, const float* q, int32_t dtype, void* G, void* ws,
                              size_t ws_bytes, void* stream);
 
+/* Both Cayley-Neumann builds of a layer in one batch: GR from qR and GP
+ * from qP (same arithmetic as poetx_cnp_build on each side).  Workspace:
+ * poetx_layer_cnp_workspace_bytes(layer). */
+size_t poetx_layer_cnp_workspace_bytes(const poetx_layer* layer);
+poetx_status poetx_layer_cnp_build(const poetx_layer* layer, void* ws, size_t ws_bytes, void* stream);
+
 /* Backward of poetx_cnp_build: given dG = dL/dG [nblk][b][b] (fp32), writes
  * dq = dL/dq [nblk][b(b-1)/2] (fp32), dq_k = dL/dQ[i][j] - dL/dQ[j][i].
  * accumulate != 0 adds to dq instead of overwriting it.  dtype names the

@@ -54,6 +54,8 @@ SIGNATURES = {
     "poetx_frame_export": (ctypes.c_int, [_LP, _VP, _VP]),
     "poetx_cnp_build": (ctypes.c_int, [_I32, _I32, _VP, _I32, _VP, _VP, _SZ, _VP]),
     "poetx_cnp_backward": (ctypes.c_int, [_I32, _I32, _VP, _VP, _VP, _I32, _I32, _VP, _SZ, _VP]),
+    "poetx_layer_cnp_workspace_bytes": (_SZ, [_LP]),
+    "poetx_layer_cnp_build": (ctypes.c_int, [_LP, _VP, _SZ, _VP]),
     "poetx_forward": (ctypes.c_int, [_LP, _I64, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "poetx_backward": (ctypes.c_int, [_LP, _I64, _VP, _VP, _VP, _VP, _VP, _VP, _I32, _VP, _SZ, _VP]),
     "poetx_merge": (ctypes.c_int, [_LP, _VP, _VP, _VP, _VP, _SZ, _VP]),
@@ -160,6 +162,15 @@ def poetx_cnp_backward(nblk: int, b: int, q, dG, dq, accumulate: int, dtype: int
                        stream=None) -> None:
     _check(lib().poetx_cnp_backward(nblk, b, _ptr(q), _ptr(dG), _ptr(dq), accumulate, dtype, _ptr(ws), ws_bytes,
                                     _stream(stream)), "poetx_cnp_backward")
+
+
+def poetx_layer_cnp_workspace_bytes(layer: poetx_layer) -> int:
+    return lib().poetx_layer_cnp_workspace_bytes(ctypes.byref(layer))
+
+
+def poetx_layer_cnp_build(layer: poetx_layer, ws, ws_bytes: int, stream=None) -> None:
+    _check(lib().poetx_layer_cnp_build(ctypes.byref(layer), _ptr(ws), ws_bytes, _stream(stream)),
+           "poetx_layer_cnp_build")
 
 
 def poetx_forward(layer: poetx_layer, T: int, x, z, y_save, ws, ws_bytes: int, stream=None) -> None:

@@ -126,4 +126,102 @@ __global__ void transpose_blocks_kernel(const T* __restrict__ in, float* __restr
   }
 }
 
+
+// ---------------------------------------------------------------------------
+// Two-sided variants: the blocks of G_R and G_P (or of any two block sets
+// with the same b) are processed as one batch [0, n0) + [n0, nblk).
+// Matrices live in row-strided block arrays: block t starts at t * bs, rows
+// ld apart (so a block can sit inside a wider concatenated row).
+
+// Unpack packed triangles into Q (and optionally a second copy); one warp
+// per triangle row.  grid.x covers nblk * b rows, 8 warps per block.
+__global__ void unpack_skew2_kernel(const float* __restrict__ q0, int n0, const float* __restrict__ q1, int nblk,
+                                    int b, float* __restrict__ o1, int64_t ld1, int64_t bs1, float* __restrict__ o2,
+                                    int64_t ld2, int64_t bs2) {
+  const int64_t row_global = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row_global >= static_cast<int64_t>(nblk) * b) return;
+  const int blk = static_cast<int>(row_global / b);
+  const int i = static_cast<int>(row_global - static_cast<int64_t>(blk) * b);
+  const int64_t L = static_cast<int64_t>(b) * (b - 1) / 2;
+  const float* qb = blk < n0 ? q0 + blk * L : q1 + (blk - n0) * L;
+  float* A1 = o1 + blk * bs1;
+  float* A2 = o2 ? o2 + blk * bs2 : nullptr;
+  const int64_t k0 = tri_index(i, i + 1, b);
+  for (int j = i + 1 + lane; j < b; j += 32) {
+    const float v = qb[k0 + (j - i - 1)];
+    A1[i * ld1 + j] = v;
+    A1[j * ld1 + i] = -v;
+    if (A2) {
+      A2[i * ld2 + j] = v;
+      A2[j * ld2 + i] = -v;
+    }
+  }
+  if (lane == 0) {
+    A1[i * ld1 + i] = 0.f;
+    if (A2) A2[i * ld2 + i] = 0.f;
+  }
+}
+
+// dG = sum over token splits of the partial products, in split order, for
+// both sides; writes dG to o1 (and o2 if given) and dG^T to ot.  32 x 32
+// tiles through shared memory: grid (b/32, b/32, nblk), block (32, 8).
+__global__ void reduce_transpose_kernel(const float* __restrict__ part0, int splits0, int n0,
+                                        const float* __restrict__ part1, int splits1, int n1, int b,
+                                        float* __restrict__ o1, int64_t ld1, int64_t bs1, float* __restrict__ o2,
+                                        int64_t ld2, int64_t bs2, float* __restrict__ ot, int64_t ldt, int64_t bst) {
+  __shared__ float tile[32][33];
+  const int t = blockIdx.z;
+  const float* part;
+  int splits;
+  int64_t sstride, off;
+  const int64_t bb = static_cast<int64_t>(b) * b;
+  if (t < n0) {
+    part = part0;
+    splits = splits0;
+    sstride = static_cast<int64_t>(n0) * bb;
+    off = t * bb;
+  } else {
+    part = part1;
+    splits = splits1;
+    sstride = static_cast<int64_t>(n1) * bb;
+    off = (t - n0) * bb;
+  }
+  const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int r = r0 + i, c = c0 + threadIdx.x;
+    if (r < b && c < b) {
+      const int64_t e = off + static_cast<int64_t>(r) * b + c;
+      float acc = part[e];
+      for (int s = 1; s < splits; ++s) acc += part[s * sstride + e];
+      o1[t * bs1 + r * ld1 + c] = acc;
+      if (o2) o2[t * bs2 + r * ld2 + c] = acc;
+      tile[i][threadIdx.x] = acc;
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int r = c0 + i, c = r0 + threadIdx.x;
+    if (r < b && c < b) ot[t * bst + r * ldt + c] = tile[threadIdx.x][i];
+  }
+}
+
+// dq[k(i,j)] (+)= dA[i][j] - dA[j][i] for both sides; one block row per
+// (blk, i).
+__global__ void fold_skew2_kernel(const float* __restrict__ dA, int64_t ld, int64_t bs, int n0, int b,
+                                  float* __restrict__ dq0, float* __restrict__ dq1, int accumulate) {
+  const int64_t row_global = blockIdx.x;
+  const int blk = static_cast<int>(row_global / b);
+  const int i = static_cast<int>(row_global - static_cast<int64_t>(blk) * b);
+  const int64_t L = static_cast<int64_t>(b) * (b - 1) / 2;
+  const float* Ab = dA + blk * bs;
+  float* qb = blk < n0 ? dq0 + blk * L : dq1 + (blk - n0) * L;
+  const int64_t k0 = tri_index(i, i + 1, b);
+  for (int j = i + 1 + threadIdx.x; j < b; j += blockDim.x) {
+    const float g = Ab[static_cast<int64_t>(i) * ld + j] - Ab[static_cast<int64_t>(j) * ld + i];
+    const int64_t k = k0 + (j - i - 1);
+    qb[k] = accumulate ? qb[k] + g : g;
+  }
+}
+
 }  // namespace poetx

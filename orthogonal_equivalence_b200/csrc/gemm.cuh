@@ -40,12 +40,31 @@ struct OutDesc {
   int64_t ld = 0;            // row stride
   int64_t batch_stride = 0;  // element offset per batch index
   int64_t split_stride = 0;  // element offset per K-split (partial sums)
+  void* ptr2 = nullptr;      // batches t >= split_batch go to ptr2 (as batch t - split_batch)
+  int split_batch = 1 << 30;
+  // 2-D view of the output for TMA tensor stores (view_rows == 0: plain
+  // stores).  Element (r, n) of batch t, split s is at view row
+  // r + t*b_row + s*s_row, column n + t*b_col.
+  int64_t view_rows = 0, view_cols = 0;
+  int b_row = 0, b_col = 0, s_row = 0;
 };
 
 struct AddDesc {
   const float* ptr = nullptr;  // fp32, indexed like the output
   int64_t ld = 0, batch_stride = 0;
   float beta = 0.f;
+};
+
+// Extra fp32 output written from the final value v of the main output:
+//   out = cv * v + ca * add,  stored at (r, n) or, transposed, at (n, r).
+struct ExtraOut {
+  float* ptr = nullptr;
+  int64_t ld = 0, batch_stride = 0;
+  float cv = 1.f;
+  const float* add = nullptr;
+  int64_t add_ld = 0, add_bs = 0;
+  float ca = 0.f;
+  int transposed = 0;
 };
 
 struct GemmDesc {
@@ -56,12 +75,15 @@ struct GemmDesc {
   float alpha = 1.f;
   AddDesc add1, add2;
   float diag = 0.f;
+  ExtraOut ex[2];
 };
 
 // ------------------------------------------------------------------ epilogue
 struct EpiParams {
   int M, N;
   void* c;
+  void* c2;
+  int c_split;
   int c_et;
   int64_t ldc, c_bs, c_ss;
   float alpha;
@@ -72,6 +94,7 @@ struct EpiParams {
   int64_t x2_ld, x2_bs;
   float beta2;
   float diag;
+  ExtraOut ex[2];
 };
 
 inline EpiParams make_epi(const GemmDesc& g) {
@@ -79,6 +102,8 @@ inline EpiParams make_epi(const GemmDesc& g) {
   e.M = g.M;
   e.N = g.N;
   e.c = g.C.ptr;
+  e.c2 = g.C.ptr2;
+  e.c_split = g.C.split_batch;
   e.c_et = g.C.et;
   e.ldc = g.C.ld;
   e.c_bs = g.C.batch_stride;
@@ -93,15 +118,42 @@ inline EpiParams make_epi(const GemmDesc& g) {
   e.x2_bs = g.add2.batch_stride;
   e.beta2 = g.add2.beta;
   e.diag = g.diag;
+  e.ex[0] = g.ex[0];
+  e.ex[1] = g.ex[1];
   return e;
 }
 
+// alpha * acc + beta1 X1 + beta2 X2 + diag I at (r, n) of batch t
 __device__ __forceinline__ float epi_value(const EpiParams& e, float acc, int t, int64_t r, int64_t n) {
   float v = e.alpha * acc;
   if (e.x1) v += e.beta1 * e.x1[t * e.x1_bs + r * e.x1_ld + n];
   if (e.x2) v += e.beta2 * e.x2[t * e.x2_bs + r * e.x2_ld + n];
   if (r == n) v += e.diag;
   return v;
+}
+
+// Element offset of the main output for batch t / split sp (and the base
+// pointer that batch goes to).
+__device__ __forceinline__ int64_t epi_out_base(const EpiParams& e, int t, int sp, void*& base) {
+  if (t >= e.c_split) {
+    base = e.c2;
+    t -= e.c_split;
+  } else {
+    base = e.c;
+  }
+  return t * e.c_bs + sp * e.c_ss;
+}
+
+// Extra outputs of one element with final value v.
+__device__ __forceinline__ void epi_extra_scalar(const EpiParams& e, int t, int64_t r, int64_t n, float v) {
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const ExtraOut& x = e.ex[k];
+    if (!x.ptr) continue;
+    float o = x.cv * v;
+    if (x.add) o += x.ca * x.add[t * x.add_bs + r * x.add_ld + n];
+    x.ptr[t * x.batch_stride + (x.transposed ? n * x.ld + r : r * x.ld + n)] = o;
+  }
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -117,6 +169,8 @@ constexpr int NUM_THREADS = 192;  // warp 0: TMA, warp 1: MMA + TMEM owner, warp
 constexpr int GROUP_M = 16;       // M-tiles per raster group (L2 reuse of the B panel)
 
 struct Params {
+  int tma_store;  // 1: the epilogue writes C through shared memory with TMA stores
+  int c_brow, c_bcol, c_srow;
   int M, N, K, batch, splits, k_per_split;
   int tiles_m, tiles_n;
   int a_mn, b_mn;
@@ -142,10 +196,12 @@ struct Cfg {
   static constexpr int A_BYTES = BM * 128;
   static constexpr int B_BYTES = BN * 128;
   static constexpr int STAGE_BYTES = B_RES ? A_BYTES : A_BYTES + B_BYTES;
-  static constexpr int STAGES = B_RES ? 5 : (BN == 256 ? 4 : (BN == 128 ? 6 : 8));
+  static constexpr int STAGES = B_RES ? 4 : (BN == 256 ? 4 : (BN == 128 ? 6 : 8));
   static constexpr int MAX_KB_RES = B_RES ? (128 * 1024) / B_BYTES : 0;  // resident K-blocks of B
   static constexpr int TMEM_COLS = 2 * BN;  // double-buffered fp32 accumulator
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + MAX_KB_RES * B_BYTES + 1024 + 256;
+  static constexpr int EPI_BOX = 32 * 128;       // one warp's 32-row x 128-byte output box
+  static constexpr int EPI_BYTES = 4 * 2 * EPI_BOX;  // 4 epilogue warps, double-buffered
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + MAX_KB_RES * B_BYTES + EPI_BYTES + 1024 + 256;
 };
 
 // Streamed mode: round-robin tiles, GROUP_M-grouped raster inside each
@@ -187,11 +243,13 @@ __device__ __forceinline__ void tile_range(int total, int& t0, int& t1, int& ste
 
 template <int BN, bool TF32, bool B_RES>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, Params p) {
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ CUtensorMap tmC, Params p) {
   using C = Cfg<BN, TF32, B_RES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES + C::MAX_KB_RES * C::B_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES + C::MAX_KB_RES * C::B_BYTES +
+                                               C::EPI_BYTES);
   // bars: full[STAGES], empty[STAGES], tfull[2], tempty[2], drain, bfull, bempty
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * C::STAGES + 7);
 
@@ -199,6 +257,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int lane = threadIdx.x & 31;
   const uint32_t smem_base = smem_u32(smem);
   const uint32_t sB_res = smem_base + C::STAGES * C::STAGE_BYTES;  // resident B (B_RES only)
+  const uint32_t sEpi = sB_res + C::MAX_KB_RES * C::B_BYTES;         // output staging boxes
   auto bar = [&](int i) { return smem_u32(bars + i); };
   const int FULL = 0, EMPTY = C::STAGES, TFULL = 2 * C::STAGES, TEMPTY = 2 * C::STAGES + 2,
             DRAIN = 2 * C::STAGES + 4, BFULL = 2 * C::STAGES + 5, BEMPTY = 2 * C::STAGES + 6;
@@ -367,6 +426,70 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_commit(bar(DRAIN));
       mbar_wait(bar(DRAIN), 0, DERR_GEMM_WAIT);
     }
+  } else if (p.tma_store) {
+    // ---------------- epilogue: TMEM -> registers -> swizzled smem box -> TMA store
+    // Each warp owns TMEM lanes [32*quarter, +32) = 32 output rows; one box is
+    // 32 rows x 128 bytes (64 bf16 or 32 fp32 columns), 128-byte swizzled:
+    // the 16-byte chunk k of row i sits at slot k ^ (i & 7).
+    const int quarter = warp & 3;
+    const EpiParams& e = p.epi;
+    const uint32_t my_boxes = sEpi + (warp - 2) * 2 * C::EPI_BOX;
+    constexpr int CHO_BF16 = 64, CHO_F32 = 32;
+    int buf = 0;
+    int local = 0;
+    for (int tile = t0; tile < t1; tile += tstep, ++local) {
+      int bt, sp, mt, nt;
+      decode_tile<B_RES>(p, tile, bt, sp, mt, nt);
+      const int acc = local & 1;
+      const uint32_t acc_phase = (local >> 1) & 1;
+      bool ok = mbar_wait(bar(TFULL + acc), acc_phase, DERR_GEMM_WAIT);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const int row0 = mt * BM + quarter * 32;
+      const bool warp_rows = row0 < e.M;  // boxes past M (a b x b block smaller than the tile) are skipped
+      const int vrow = row0 + bt * p.c_brow + sp * p.c_srow;
+      const int cho = e.c_et == ET_BF16 ? CHO_BF16 : CHO_F32;
+      const uint32_t tl = tmem_base + acc * BN + (static_cast<uint32_t>(quarter * 32) << 16);
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += cho) {
+        uint32_t w[32];  // one 128-byte output row of this lane
+        if (e.c_et == ET_BF16) {
+          float v[32];
+          tmem_ld_32cols(tl + c0, v);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(e.alpha * v[2 * i], e.alpha * v[2 * i + 1]);
+          tmem_ld_32cols(tl + c0 + 32, v);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) w[16 + i] = pack_bf16x2(e.alpha * v[2 * i], e.alpha * v[2 * i + 1]);
+        } else {
+          float v[32];
+          tmem_ld_32cols(tl + c0, v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(e.alpha * v[i]);
+        }
+        if (!warp_rows) continue;
+        if (lane == 0) bulk_wait_read<1>();  // the store that last used this box has read it
+        __syncwarp();
+        const uint32_t box = my_boxes + buf * C::EPI_BOX;
+        const uint32_t rowp = box + lane * 128;
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(rowp + ((k ^ (lane & 7)) << 4)),
+                       "r"(w[4 * k]), "r"(w[4 * k + 1]), "r"(w[4 * k + 2]), "r"(w[4 * k + 3])
+                       : "memory");
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tmC, box, nt * BN + c0 + bt * p.c_bcol, vrow);
+          bulk_commit();
+        }
+        buf ^= 1;
+      }
+      tc_fence_before();
+      mbar_arrive(bar(TEMPTY + acc));
+    }
+    if (lane == 0) bulk_wait_all();
   } else {
     // ---------------- epilogue: TMEM -> registers -> global
     const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter + 32)
@@ -383,7 +506,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const int64_t r = static_cast<int64_t>(mt) * BM + quarter * 32 + lane;
       const bool row_ok = r < e.M;
-      const int64_t obase = bt * e.c_bs + sp * e.c_ss + r * e.ldc;
+      void* cbase;
+      const int64_t obase = epi_out_base(e, bt, sp, cbase) + r * e.ldc;
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 32) {
         float v[32];
@@ -423,23 +547,57 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               if (r == n0 + i) v[i] += e.diag;
           }
           if (e.c_et == ET_BF16) {
-            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(e.c) + obase + n0);
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(cbase) + obase + n0);
 #pragma unroll
             for (int q = 0; q < 4; ++q)
               dst[q] = make_uint4(pack_bf16x2(v[8 * q + 0], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
                                   pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
           } else {
-            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(e.c) + obase + n0);
+            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(cbase) + obase + n0);
 #pragma unroll
             for (int q = 0; q < 8; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
           }
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const ExtraOut& x = e.ex[k];
+            if (!x.ptr) continue;
+            float o[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = x.cv * v[i];
+            if (x.add) {
+              const float4* ap = reinterpret_cast<const float4*>(x.add + bt * x.add_bs + r * x.add_ld + n0);
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                const float4 a = __ldg(ap + q);
+                o[4 * q] += x.ca * a.x;
+                o[4 * q + 1] += x.ca * a.y;
+                o[4 * q + 2] += x.ca * a.z;
+                o[4 * q + 3] += x.ca * a.w;
+              }
+            }
+            if (x.transposed) {
+              // lanes hold consecutive rows r: each column n is one coalesced 128-byte row segment
+              float* dst = x.ptr + bt * x.batch_stride + n0 * x.ld + r;
+#pragma unroll
+              for (int i = 0; i < 32; ++i) dst[i * x.ld] = o[i];
+            } else {
+              float4* dst = reinterpret_cast<float4*>(x.ptr + bt * x.batch_stride + r * x.ld + n0);
+#pragma unroll
+              for (int q = 0; q < 8; ++q) dst[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+            }
+          }
         } else {
-          for (int i = 0; i < 32 && n0 + i < e.N; ++i) {
-            const float o = epi_value(e, v[i], bt, r, n0 + i);
-            if (e.c_et == ET_BF16)
-              reinterpret_cast<__nv_bfloat16*>(e.c)[obase + n0 + i] = __float2bfloat16_rn(o);
-            else
-              reinterpret_cast<float*>(e.c)[obase + n0 + i] = o;
+          // ragged last chunk: element by element (fully unrolled so v stays in registers)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            if (n0 + i < e.N) {
+              const float o = epi_value(e, v[i], bt, r, n0 + i);
+              if (e.c_et == ET_BF16)
+                reinterpret_cast<__nv_bfloat16*>(cbase)[obase + n0 + i] = __float2bfloat16_rn(o);
+              else
+                reinterpret_cast<float*>(cbase)[obase + n0 + i] = o;
+              epi_extra_scalar(e, bt, r, n0 + i, o);
+            }
           }
         }
       }
@@ -539,11 +697,13 @@ __global__ void __launch_bounds__(THREADS) gemm_kernel(Params p) {
       const int64_t n = n0 + tx * 4 + j;
       if (n >= e.N) continue;
       const float v = epi_value(e, acc[i][j], t, r, n);
-      const int64_t o = t * e.c_bs + sp * e.c_ss + r * e.ldc + n;
+      void* cbase;
+      const int64_t o = epi_out_base(e, t, sp, cbase) + r * e.ldc + n;
       if (e.c_et == ET_BF16)
-        reinterpret_cast<__nv_bfloat16*>(e.c)[o] = __float2bfloat16_rn(v);
+        reinterpret_cast<__nv_bfloat16*>(cbase)[o] = __float2bfloat16_rn(v);
       else
-        reinterpret_cast<float*>(e.c)[o] = v;
+        reinterpret_cast<float*>(cbase)[o] = v;
+      epi_extra_scalar(e, t, r, n, v);
     }
   }
 }

@@ -66,9 +66,16 @@ cudaError_t launch_tc_typed(const GemmDesc& g, cudaStream_t st, int device) {
   if (!vec_ok(g.add1) || !vec_ok(g.add2)) return cudaErrorInvalidValue;
   {
     const int v = g.C.et == ET_BF16 ? 8 : 4;
-    if ((reinterpret_cast<uintptr_t>(g.C.ptr) & 15u) != 0 || g.C.ld % v != 0 || g.C.batch_stride % v != 0 ||
-        g.C.split_stride % v != 0)
+    if ((reinterpret_cast<uintptr_t>(g.C.ptr) & 15u) != 0 || (reinterpret_cast<uintptr_t>(g.C.ptr2) & 15u) != 0 ||
+        g.C.ld % v != 0 || g.C.batch_stride % v != 0 || g.C.split_stride % v != 0)
       return cudaErrorInvalidValue;
+    for (const ExtraOut& x : g.ex) {
+      if (!x.ptr) continue;
+      if ((reinterpret_cast<uintptr_t>(x.ptr) & 15u) != 0 || x.ld % 4 != 0 || x.batch_stride % 4 != 0)
+        return cudaErrorInvalidValue;
+      if (x.add && ((reinterpret_cast<uintptr_t>(x.add) & 15u) != 0 || x.add_ld % 4 != 0 || x.add_bs % 4 != 0))
+        return cudaErrorInvalidValue;
+    }
   }
   static bool attr_set[64] = {false};
   if (device >= 0 && device < 64 && !attr_set[device]) {
@@ -77,10 +84,34 @@ cudaError_t launch_tc_typed(const GemmDesc& g, cudaStream_t st, int device) {
     if (e != cudaSuccess) return e;
     attr_set[device] = true;
   }
-  CUtensorMap ma, mb;
+  CUtensorMap ma, mb, mc;
   if (!encode_map(&ma, g.A, g.A.mn_major ? C::CH : tc::BM)) return cudaErrorInvalidValue;
   if (!encode_map(&mb, g.B, g.B.mn_major ? C::CH : BN)) return cudaErrorInvalidValue;
   tc::Params p;
+  // TMA-store epilogue: plain output (no addends, extra outputs, split pointer
+  // or diagonal) described by a 2-D view; boxes of 32 rows x 128 bytes.
+  const int c_esz = elem_size(g.C.et);
+  const bool plain_out = g.C.view_rows > 0 && !g.add1.ptr && !g.add2.ptr && !g.ex[0].ptr && !g.ex[1].ptr &&
+                         !g.C.ptr2 && g.diag == 0.f;
+  // rows past M inside a 32-row box must fall outside the view (TMA clips
+  // them) unless M is a whole number of boxes
+  const bool rows_ok = g.M % 32 == 0 || (g.C.b_row == 0 && g.C.s_row == 0 && g.M == g.C.view_rows);
+  p.tma_store = plain_out && rows_ok && (reinterpret_cast<uintptr_t>(g.C.ptr) & 15u) == 0 &&
+                (g.C.ld * c_esz) % 16 == 0;
+  p.c_brow = g.C.b_row;
+  p.c_bcol = g.C.b_col;
+  p.c_srow = g.C.s_row;
+  if (p.tma_store) {
+    Operand2D cv;
+    cv.ptr = g.C.ptr;
+    cv.et = g.C.et;
+    cv.rows = g.C.view_rows;
+    cv.cols = g.C.view_cols;
+    cv.ld = g.C.ld;
+    if (!encode_map(&mc, cv, 32)) return cudaErrorInvalidValue;
+  } else {
+    mc = ma;  // unused
+  }
   p.M = g.M;
   p.N = g.N;
   p.K = g.K;
@@ -113,7 +144,7 @@ cudaError_t launch_tc_typed(const GemmDesc& g, cudaStream_t st, int device) {
   const int grid = total < sm_count(device) ? total : sm_count(device);
   if (grid <= 0) return cudaSuccess;
   if (B_RES && p.k_per_split > C::MAX_KB_RES * C::CH) return cudaErrorInvalidValue;
-  tc::gemm_kernel<BN, TF32, B_RES><<<grid, tc::NUM_THREADS, C::SMEM_BYTES, st>>>(ma, mb, p);
+  tc::gemm_kernel<BN, TF32, B_RES><<<grid, tc::NUM_THREADS, C::SMEM_BYTES, st>>>(ma, mb, mc, p);
   return cudaGetLastError();
 }
 

@@ -190,8 +190,11 @@ int dg_splits(int nblk, int b, int64_t T, int32_t dtype) {
   return static_cast<int>(s);
 }
 
-size_t cnp_build_ws(int32_t nblk, int32_t b) { return 3 * al(sizeof(float) * size_t(nblk) * b * b); }
-size_t cnp_bwd_ws(int32_t nblk, int32_t b) { return 9 * al(sizeof(float) * size_t(nblk) * b * b); }
+// Scratch of the CNP build (3 b x b arrays per block) and backward (11).
+size_t cnp_bwd_ws(int32_t nblk, int32_t b) {
+  const size_t u = sizeof(float) * size_t(nblk) * b * b;
+  return al(2 * u) + al(2 * u) + al(3 * u) + al(3 * u) + al(u);
+}
 
 size_t fwd_ws(const poetx_layer* L, int64_t T) {
   const size_t es = dtype_size(L->dtype);
@@ -202,12 +205,10 @@ size_t bwd_ws(const poetx_layer* L, int64_t T) {
   const size_t es = dtype_size(L->dtype);
   const int64_t mx = L->m > L->n ? L->m : L->n;
   const int nR = L->m / L->b, nP = L->n / L->b;
-  const int nmax = nR > nP ? nR : nP;
   const size_t bb = size_t(L->b) * L->b;
   return kAlign + 2 * al(es * T * mx) + al(es * T * L->m) +
          al(sizeof(float) * dg_splits(nP, L->b, T, L->dtype) * nP * bb) +
-         al(sizeof(float) * dg_splits(nR, L->b, T, L->dtype) * nR * bb) + al(sizeof(float) * nmax * bb) +
-         cnp_bwd_ws(nmax, L->b);
+         al(sizeof(float) * dg_splits(nR, L->b, T, L->dtype) * nR * bb) + cnp_bwd_ws(nR + nP, L->b);
 }
 
 size_t merge_ws(const poetx_layer* L) {
@@ -381,6 +382,9 @@ GemmDesc blockdiag_desc(const void* in, int et_in, int64_t T, int d, int b, cons
   g.C.et = et_out;
   g.C.ld = d;
   g.C.batch_stride = b;
+  g.C.view_rows = T;
+  g.C.view_cols = d;
+  g.C.b_col = b;
   return g;
 }
 
@@ -411,36 +415,11 @@ GemmDesc blockgrad_desc(const void* in1, const void* in2, int et, int64_t T, int
   g.C.ld = b;
   g.C.batch_stride = int64_t(b) * b;
   g.C.split_stride = int64_t(d / b) * b * b;
+  g.C.view_rows = int64_t(splits) * (d / b) * b;
+  g.C.view_cols = b;
+  g.C.b_row = b;
+  g.C.s_row = (d / b) * b;
   return g;
-}
-
-// Square b x b products over nblk blocks of fp32 scratch, in "NT" form:
-//   C_t = alpha * X_t Y_t^T   (both operands K-major)
-// Every tf32 product is written this way (tcgen05 tf32 reads K-major tiles of
-// the 128-byte swizzle; the MN-major fp32 tile layout is not used).
-GemmDesc nt_desc(const float* X, const float* Y, int nblk, int b, void* out, int et_out, float alpha = 1.f) {
-  GemmDesc g;
-  g.M = b;
-  g.N = b;
-  g.K = b;
-  g.batch = nblk;
-  g.A = blocks_view(X, ET_F32, nblk, b, true);  // A(i, k) = X[i][k]
-  g.B = blocks_view(Y, ET_F32, nblk, b, true);  // B(k, n) = Y[n][k]
-  g.C.ptr = out;
-  g.C.et = et_out;
-  g.C.ld = b;
-  g.C.batch_stride = int64_t(b) * b;
-  g.alpha = alpha;
-  return g;
-}
-
-AddDesc add_blocks(const float* p, int b, float beta) {
-  AddDesc a;
-  a.ptr = p;
-  a.ld = b;
-  a.batch_stride = int64_t(b) * b;
-  a.beta = beta;
-  return a;
 }
 
 // ---------------------------------------------------------------- CNP
@@ -449,80 +428,170 @@ AddDesc add_blocks(const float* p, int b, float beta) {
 //   S   = Q Q    = -(Q Q^T)
 //   H S = H S^T                       (H = 2Q + S)
 //   G   = I + 2Q + 2S + H S           (= (I+Q)(I+Q+Q^2+Q^3))
-poetx_status cnp_build_impl(int32_t nblk, int32_t b, const float* q, int32_t dtype, void* G, Carver& ws,
-                            cudaStream_t st, int device) {
+// Both sides of a layer (the G_R and G_P blocks) run as one batch of
+// n0 + n1 blocks.
+
+// View of a block array whose block t starts at p + t*b*ld (b rows, ld apart),
+// using its first kcols columns as the K dimension (K-major).
+Operand2D cat_view(const float* p, int nblk, int b, int64_t ld, int kcols) {
+  Operand2D o;
+  o.ptr = p;
+  o.et = ET_F32;
+  o.rows = int64_t(nblk) * b;
+  o.cols = kcols;
+  o.ld = ld;
+  o.mn_major = false;
+  o.b_row = b;
+  o.b_col = 0;
+  return o;
+}
+
+GemmDesc cat_nt_desc(const float* X, const float* Y, int nblk, int b, int64_t ld, int kcols, float alpha) {
+  GemmDesc g;
+  g.M = b;
+  g.N = b;
+  g.K = kcols;
+  g.batch = nblk;
+  g.A = cat_view(X, nblk, b, ld, kcols);
+  g.B = cat_view(Y, nblk, b, ld, kcols);
+  g.alpha = alpha;
+  return g;
+}
+
+OutDesc out_blocks(void* p, int et, int b, int64_t ld) {
+  OutDesc o;
+  o.ptr = p;
+  o.et = et;
+  o.ld = ld;
+  o.batch_stride = int64_t(b) * ld;
+  return o;
+}
+
+AddDesc add_view(const float* p, int b, int64_t ld, float beta) {
+  AddDesc a;
+  a.ptr = p;
+  a.ld = ld;
+  a.batch_stride = int64_t(b) * ld;
+  a.beta = beta;
+  return a;
+}
+
+ExtraOut extra_out(float* p, int b, int64_t ld, float cv, bool transposed) {
+  ExtraOut x;
+  x.ptr = p;
+  x.ld = ld;
+  x.batch_stride = int64_t(b) * ld;
+  x.cv = cv;
+  x.transposed = transposed ? 1 : 0;
+  return x;
+}
+
+size_t cnp_units(int32_t nblk, int32_t b) { return al(sizeof(float) * size_t(nblk) * b * b); }
+
+// G0 (n0 blocks) from q0 and G1 (n1 blocks) from q1.
+poetx_status cnp_build2(int32_t b, int32_t dtype, const float* q0, int n0, void* G0, const float* q1, int n1,
+                        void* G1, Carver& ws, cudaStream_t st, int device) {
+  const int nblk = n0 + n1;
   const size_t nbb = size_t(nblk) * b * b;
   float* Q = ws.take<float>(sizeof(float) * nbb);
   float* S = ws.take<float>(sizeof(float) * nbb);
   float* H = ws.take<float>(sizeof(float) * nbb);
   const bool tc_path = use_tc(dtype);
+  const int64_t bb = int64_t(b) * b;
   PROFILED(ST_CNP_ELEM, st,
-           unpack_skew_kernel<<<static_cast<int>((int64_t(nblk) * b + 7) / 8), 256, 0, st>>>(q, nblk, b, Q));
+           unpack_skew2_kernel<<<static_cast<int>((int64_t(nblk) * b + 7) / 8), 256, 0, st>>>(
+               q0, n0, q1, nblk, b, Q, b, bb, nullptr, 0, 0));
   POETX_CUDA(cudaGetLastError());
-  PROFILED(ST_CNP_GEMM, st, POETX_CUDA(launch_gemm(nt_desc(Q, Q, nblk, b, S, ET_F32, -1.f), tc_path, st, device)));
-  PROFILED(ST_CNP_ELEM, st, axpby_kernel<<<grid_for(nbb, 256, device), 256, 0, st>>>(Q, 2.f, S, 1.f, H, nbb));
-  POETX_CUDA(cudaGetLastError());
-  GemmDesc g = nt_desc(H, S, nblk, b, G, elem_type(dtype));
-  g.add1 = add_blocks(Q, b, 2.f);
-  g.add2 = add_blocks(S, b, 2.f);
-  g.diag = 1.f;
-  PROFILED(ST_CNP_GEMM, st, POETX_CUDA(launch_gemm(g, tc_path, st, device)));
+  // S = -(Q Q^T); H = S + 2Q as a second output
+  {
+    GemmDesc g = cat_nt_desc(Q, Q, nblk, b, b, b, -1.f);
+    g.C = out_blocks(S, ET_F32, b, b);
+    g.ex[0] = extra_out(H, b, b, 1.f, false);
+    g.ex[0].add = Q;
+    g.ex[0].add_ld = b;
+    g.ex[0].add_bs = bb;
+    g.ex[0].ca = 2.f;
+    PROFILED(ST_CNP_GEMM, st, POETX_CUDA(launch_gemm(g, tc_path, st, device)));
+  }
+  // G = H S^T + 2Q + 2S + I  (S^T = S)
+  {
+    GemmDesc g = cat_nt_desc(H, S, nblk, b, b, b, 1.f);
+    g.C = out_blocks(G0, elem_type(dtype), b, b);
+    g.C.ptr2 = G1;
+    g.C.split_batch = n0;
+    g.add1 = add_view(Q, b, b, 2.f);
+    g.add2 = add_view(S, b, b, 2.f);
+    g.diag = 1.f;
+    PROFILED(ST_CNP_GEMM, st, POETX_CUDA(launch_gemm(g, tc_path, st, device)));
+  }
   return POETX_OK;
 }
 
 // dq from dG for G = I + 2A + 2S + H S with S = A A, H = 2A + S:
 //   dH = dG S^T;  dS = 2 dG + H^T dG + dH;  dA = 2 dG + 2 dH + dS A^T + A^T dS;
 //   dq_k = dA[i][j] - dA[j][i].
-// In X Y^T form: H^T dG = (H^T)(dG^T)^T, A^T dS = -(A)(dS^T)^T.
-poetx_status cnp_backward_impl(int32_t nblk, int32_t b, const float* q, const float* dG, float* dq,
-                               int32_t accumulate, int32_t dtype, Carver& ws, cudaStream_t st, int device) {
+// Written as three X Y^T products over concatenated K (A^T = -A):
+//   S  = -(A A^T)
+//   dS = 2 dG + [H^T | dG] [dG^T | S]^T
+//   dA = 2 dG + [dS | A | dG] [A | -dS^T | 2S]^T
+// The concatenated operands X1 = [H^T | dG], Y1 = [dG^T | S] (b x 2b blocks)
+// and X2 = [dS | A | dG], Y2 = [A | -dS^T | 2S] (b x 3b blocks) are filled
+// in place by the unpack, the split reduction and the GEMM epilogues.
+// dG of side k is the sum of splits_k partial arrays part_k.
+poetx_status cnp_backward2(int32_t b, int32_t dtype, const float* q0, int n0, const float* part0, int splits0,
+                           float* dq0, const float* q1, int n1, const float* part1, int splits1, float* dq1,
+                           int32_t accumulate, Carver& ws, cudaStream_t st, int device) {
+  const int nblk = n0 + n1;
   const size_t nbb = size_t(nblk) * b * b;
-  float* A = ws.take<float>(sizeof(float) * nbb);
-  float* S = ws.take<float>(sizeof(float) * nbb);
-  float* H = ws.take<float>(sizeof(float) * nbb);
-  float* Ht = ws.take<float>(sizeof(float) * nbb);
-  float* dGt = ws.take<float>(sizeof(float) * nbb);
-  float* dH = ws.take<float>(sizeof(float) * nbb);
-  float* dS = ws.take<float>(sizeof(float) * nbb);
-  float* dSt = ws.take<float>(sizeof(float) * nbb);
-  float* T1 = ws.take<float>(sizeof(float) * nbb);
-  float* dA = H;  // H is dead once Ht exists
+  const int64_t b2 = 2 * int64_t(b), b3 = 3 * int64_t(b);
+  float* X1 = ws.take<float>(sizeof(float) * 2 * nbb);
+  float* Y1 = ws.take<float>(sizeof(float) * 2 * nbb);
+  float* X2 = ws.take<float>(sizeof(float) * 3 * nbb);
+  float* Y2 = ws.take<float>(sizeof(float) * 3 * nbb);
+  float* dA = ws.take<float>(sizeof(float) * nbb);
   const bool tc_path = use_tc(dtype);
-  const dim3 tgrid((b + 31) / 32, (b + 31) / 32, nblk), tblock(32, 8);
+  // A -> X2[:, b:2b] and Y2[:, 0:b]
   PROFILED(ST_CNP_ELEM, st,
-           unpack_skew_kernel<<<static_cast<int>((int64_t(nblk) * b + 7) / 8), 256, 0, st>>>(q, nblk, b, A));
-  POETX_CUDA(cudaGetLastError());
-  PROFILED(ST_CNP_GEMM, st, POETX_CUDA(launch_gemm(nt_desc(A, A, nblk, b, S, ET_F32, -1.f), tc_path, st, device)));
-  PROFILED(ST_CNP_ELEM, st, axpby_kernel<<<grid_for(nbb, 256, device), 256, 0, st>>>(A, 2.f, S, 1.f, H, nbb));
-  PROFILED(ST_CNP_ELEM, st, transpose_blocks_kernel<<<tgrid, tblock, 0, st>>>(H, Ht, b));
-  PROFILED(ST_CNP_ELEM, st, transpose_blocks_kernel<<<tgrid, tblock, 0, st>>>(dG, dGt, b));
-  POETX_CUDA(cudaGetLastError());
-  // dH = dG S^T
-  PROFILED(ST_CNP_GEMM, st, POETX_CUDA(launch_gemm(nt_desc(dG, S, nblk, b, dH, ET_F32), tc_path, st, device)));
-  // dS = H^T dG + 2 dG + dH
+           unpack_skew2_kernel<<<static_cast<int>((int64_t(nblk) * b + 7) / 8), 256, 0, st>>>(
+               q0, n0, q1, nblk, b, X2 + b, b3, b * b3, Y2, b3, b * b3));
+  // dG -> X1[:, b:2b], X2[:, 2b:3b];  dG^T -> Y1[:, 0:b]
   {
-    GemmDesc g = nt_desc(Ht, dGt, nblk, b, dS, ET_F32);
-    g.add1 = add_blocks(dG, b, 2.f);
-    g.add2 = add_blocks(dH, b, 1.f);
+    const dim3 grid((b + 31) / 32, (b + 31) / 32, nblk), block(32, 8);
+    PROFILED(ST_CNP_ELEM, st,
+             reduce_transpose_kernel<<<grid, block, 0, st>>>(part0, splits0, n0, part1, splits1, n1, b, X1 + b, b2,
+                                                             b * b2, X2 + 2 * b, b3, b * b3, Y1, b2, b * b2));
+  }
+  POETX_CUDA(cudaGetLastError());
+  // S = -(A A^T) -> Y1[:, b:2b];  H^T = (S + 2A)^T -> X1[:, 0:b];  2S -> Y2[:, 2b:3b]
+  {
+    GemmDesc g = cat_nt_desc(X2 + b, X2 + b, nblk, b, b3, b, -1.f);
+    g.C = out_blocks(Y1 + b, ET_F32, b, b2);
+    g.ex[0] = extra_out(X1, b, b2, 1.f, true);
+    g.ex[0].add = X2 + b;
+    g.ex[0].add_ld = b3;
+    g.ex[0].add_bs = b * b3;
+    g.ex[0].ca = 2.f;
+    g.ex[1] = extra_out(Y2 + 2 * b, b, b3, 2.f, false);
     PROFILED(ST_CNP_GEMM, st, POETX_CUDA(launch_gemm(g, tc_path, st, device)));
   }
-  PROFILED(ST_CNP_ELEM, st, transpose_blocks_kernel<<<tgrid, tblock, 0, st>>>(dS, dSt, b));
-  POETX_CUDA(cudaGetLastError());
-  // T1 = dS A^T + 2 dG + 2 dH
+  // dS = 2 dG + X1 Y1^T -> X2[:, 0:b];  -dS^T -> Y2[:, b:2b]
   {
-    GemmDesc g = nt_desc(dS, A, nblk, b, T1, ET_F32);
-    g.add1 = add_blocks(dG, b, 2.f);
-    g.add2 = add_blocks(dH, b, 2.f);
+    GemmDesc g = cat_nt_desc(X1, Y1, nblk, b, b2, 2 * b, 1.f);
+    g.C = out_blocks(X2, ET_F32, b, b3);
+    g.add1 = add_view(X1 + b, b, b2, 2.f);
+    g.ex[0] = extra_out(Y2 + b, b, b3, -1.f, true);
     PROFILED(ST_CNP_GEMM, st, POETX_CUDA(launch_gemm(g, tc_path, st, device)));
   }
-  // dA = A^T dS + T1 = -(A dS^T^T) + T1
+  // dA = 2 dG + X2 Y2^T
   {
-    GemmDesc g = nt_desc(A, dSt, nblk, b, dA, ET_F32, -1.f);
-    g.add1 = add_blocks(T1, b, 1.f);
+    GemmDesc g = cat_nt_desc(X2, Y2, nblk, b, b3, 3 * b, 1.f);
+    g.C = out_blocks(dA, ET_F32, b, b);
+    g.add1 = add_view(X2 + 2 * b, b, b3, 2.f);
     PROFILED(ST_CNP_GEMM, st, POETX_CUDA(launch_gemm(g, tc_path, st, device)));
   }
   PROFILED(ST_CNP_ELEM, st,
-           fold_skew_kernel<<<static_cast<int>(int64_t(nblk) * b), 128, 0, st>>>(dA, nblk, b, dq, accumulate));
+           fold_skew2_kernel<<<static_cast<int>(int64_t(nblk) * b), 128, 0, st>>>(dA, b, int64_t(b) * b, n0, b, dq0,
+                                                                                   dq1, accumulate));
   POETX_CUDA(cudaGetLastError());
   return POETX_OK;
 }
@@ -565,6 +634,22 @@ size_t poetx_cnp_workspace_bytes(int32_t nblk, int32_t b, int32_t dtype) {
   (void)dtype;
   if (nblk <= 0 || b < 2) return 0;
   return kAlign + cnp_bwd_ws(nblk, b);
+}
+
+size_t poetx_layer_cnp_workspace_bytes(const poetx_layer* layer) {
+  if (check_layer(layer) != POETX_OK) return 0;
+  return kAlign + cnp_bwd_ws(layer->m / layer->b + layer->n / layer->b, layer->b);
+}
+
+poetx_status poetx_layer_cnp_build(const poetx_layer* layer, void* ws, size_t ws_bytes, void* stream) {
+  POETX_TRY(check_layer(layer));
+  if (!ws || ws_bytes < poetx_layer_cnp_workspace_bytes(layer)) return POETX_E_WORKSPACE;
+  int dev;
+  POETX_TRY(current_device(&dev));
+  const poetx_layer& L = *layer;
+  Carver c(ws, ws_bytes);
+  return cnp_build2(L.b, L.dtype, L.qR, L.m / L.b, L.GR, L.qP, L.n / L.b, L.GP, c, static_cast<cudaStream_t>(stream),
+                    dev);
 }
 
 size_t poetx_forward_workspace_bytes(const poetx_layer* layer, int64_t T) {
@@ -622,7 +707,7 @@ poetx_status poetx_cnp_build(int32_t nblk, int32_t b, const float* q, int32_t dt
   int dev;
   POETX_TRY(current_device(&dev));
   Carver c(ws, ws_bytes);
-  return cnp_build_impl(nblk, b, q, dtype, G, c, static_cast<cudaStream_t>(stream), dev);
+  return cnp_build2(b, dtype, q, nblk, G, nullptr, 0, nullptr, c, static_cast<cudaStream_t>(stream), dev);
 }
 
 poetx_status poetx_cnp_backward(int32_t nblk, int32_t b, const float* q, const float* dG, float* dq,
@@ -637,7 +722,8 @@ poetx_status poetx_cnp_backward(int32_t nblk, int32_t b, const float* q, const f
   int dev;
   POETX_TRY(current_device(&dev));
   Carver c(ws, ws_bytes);
-  return cnp_backward_impl(nblk, b, q, dG, dq, accumulate, dtype, c, static_cast<cudaStream_t>(stream), dev);
+  return cnp_backward2(b, dtype, q, nblk, dG, 1, dq, nullptr, 0, nullptr, 1, nullptr, accumulate, c,
+                       static_cast<cudaStream_t>(stream), dev);
 }
 
 poetx_status poetx_forward(const poetx_layer* layer, int64_t T, const void* x, void* z, void* y_save, void* ws,
@@ -684,6 +770,8 @@ poetx_status poetx_forward(const poetx_layer* layer, int64_t T, const void* x, v
     g.C.ptr = Y;
     g.C.et = et;
     g.C.ld = L.n;
+    g.C.view_rows = T;
+    g.C.view_cols = L.n;
     PROFILED(ST_W0, st, POETX_CUDA(launch_gemm(g, tc_path, st, dev)));
   }
   // V_j = Y_j G_Pj
@@ -730,7 +818,6 @@ poetx_status poetx_backward(const poetx_layer* layer, int64_t T, const void* x, 
   void* dU = c.take<uint8_t>(es * T * L.m);
   float* partP = c.take<float>(sizeof(float) * sP * nP * bb);
   float* partR = c.take<float>(sizeof(float) * sR * nR * bb);
-  float* dG = c.take<float>(sizeof(float) * (nR > nP ? nR : nP) * bb);
 
   // dV = dz Psi_P^T
   void* dV = bufA;
@@ -758,6 +845,8 @@ poetx_status poetx_backward(const poetx_layer* layer, int64_t T, const void* x, 
     g.C.ptr = dU;
     g.C.et = et;
     g.C.ld = L.m;
+    g.C.view_rows = T;
+    g.C.view_cols = L.m;
     PROFILED(ST_W0, st, POETX_CUDA(launch_gemm(g, tc_path, st, dev)));
   }
   // Xg = x Psi_R^T (re-gathered; dV is dead)
@@ -770,21 +859,9 @@ poetx_status poetx_backward(const poetx_layer* layer, int64_t T, const void* x, 
   PROFILED(ST_DG, st, POETX_CUDA(launch_gemm(blockgrad_desc(Xg, dU, et, T, L.m, L.b, sR, partR), tc_path, st, dev)));
   // dx = dXg Psi_R
   if (dx) PROFILED(ST_PERMUTE, st, POETX_CUDA(permute_dt(L.dtype, dXg, dx, T, L.m, L.permR, 1, st, dev)));
-  // dq from dG (fixed-order reduction of the token splits, then the CNP backward)
-  PROFILED(ST_REDUCE, st,
-           reduce_splits_kernel<<<grid_for(nP * bb / 4 + 1, 256, dev), 256, 0, st>>>(partP, sP, int64_t(nP) * bb, dG));
-  POETX_CUDA(cudaGetLastError());
-  {
-    Carver c2 = c;
-    POETX_TRY(cnp_backward_impl(nP, L.b, L.qP, dG, dqP, accumulate, L.dtype, c2, st, dev));
-  }
-  PROFILED(ST_REDUCE, st,
-           reduce_splits_kernel<<<grid_for(nR * bb / 4 + 1, 256, dev), 256, 0, st>>>(partR, sR, int64_t(nR) * bb, dG));
-  POETX_CUDA(cudaGetLastError());
-  {
-    Carver c2 = c;
-    POETX_TRY(cnp_backward_impl(nR, L.b, L.qR, dG, dqR, accumulate, L.dtype, c2, st, dev));
-  }
+  // dq from the dG partial sums of both sides (fixed-order reduction of the
+  // token splits inside the CNP backward)
+  POETX_TRY(cnp_backward2(L.b, L.dtype, L.qP, nP, partP, sP, dqP, L.qR, nR, partR, sR, dqR, accumulate, c, st, dev));
   return POETX_OK;
 }
 
@@ -834,6 +911,9 @@ poetx_status poetx_merge(const poetx_layer* layer, const int32_t* new_permR, con
     g.C.et = ET_F32;
     g.C.ld = L.n;
     g.C.batch_stride = int64_t(L.b) * L.n;
+    g.C.view_rows = L.m;
+    g.C.view_cols = L.n;
+    g.C.b_row = L.b;
     PROFILED(ST_MERGE, st, POETX_CUDA(launch_gemm(g, tc_path, st, dev)));
   }
   // pass 2: At[jb + r][c] = sum_k G_Pj[k][r] B1t[c][jb + k]  (G_Pj^T, fp32, K-major)
@@ -857,6 +937,9 @@ poetx_status poetx_merge(const poetx_layer* layer, const int32_t* new_permR, con
     g.C.et = ET_F32;
     g.C.ld = L.m;
     g.C.batch_stride = int64_t(L.b) * L.m;
+    g.C.view_rows = L.n;
+    g.C.view_cols = L.m;
+    g.C.b_row = L.b;
     PROFILED(ST_MERGE, st, POETX_CUDA(launch_gemm(g, tc_path, st, dev)));
   }
   // New frame: W'[j'][i'] = At[sigP[j']][sigR[i']], sig = perm_old^-1 o perm_new.

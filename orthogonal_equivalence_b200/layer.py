@@ -13,8 +13,8 @@ from typing import Optional, Tuple
 import torch
 
 from . import (POETX_BF16, POETX_FP32, make_layer, poetx_backward, poetx_backward_workspace_bytes,
-               poetx_cnp_build, poetx_cnp_workspace_bytes, poetx_forward, poetx_forward_workspace_bytes,
-               poetx_frame_export, poetx_frame_import, poetx_merge, poetx_merge_workspace_bytes)
+               poetx_forward, poetx_forward_workspace_bytes, poetx_frame_export, poetx_frame_import,
+               poetx_layer_cnp_build, poetx_layer_cnp_workspace_bytes, poetx_merge, poetx_merge_workspace_bytes)
 
 _TORCH_DTYPE = {POETX_BF16: torch.bfloat16, POETX_FP32: torch.float32}
 
@@ -71,12 +71,11 @@ class PoetxLinear:
         return out
 
     def build(self, stream=None) -> None:
-        """G_R, G_P from qR, qP (Cayley-Neumann)."""
-        nR, nP = self.m // self.b, self.n // self.b
-        nb = poetx_cnp_workspace_bytes(max(nR, nP), self.b, self.dtype)
+        """G_R, G_P from qR, qP (Cayley-Neumann), both sides in one batch."""
+        L = self.abi()
+        nb = poetx_layer_cnp_workspace_bytes(L)
         ws = self.workspace("cnp", nb)
-        poetx_cnp_build(nR, self.b, self.qR, self.dtype, self.GR, ws, nb, stream)
-        poetx_cnp_build(nP, self.b, self.qP, self.dtype, self.GP, ws, nb, stream)
+        poetx_layer_cnp_build(L, ws, nb, stream)
 
     # -------------------------------------------------------------- layer
     def forward(self, x: torch.Tensor, save: bool = True, z: Optional[torch.Tensor] = None,
