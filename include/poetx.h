@@ -115,6 +115,23 @@ poetx_status poetx_cnp_build(int32_t nblk, int32_t b, const float* q, int32_t dt
 size_t poetx_layer_cnp_workspace_bytes(const poetx_layer* layer);
 poetx_status poetx_layer_cnp_build(const poetx_layer* layer, void* ws, size_t ws_bytes, void* stream);
 
+/* poetx_cnp_build without a caller workspace, for callers that cannot
+ * allocate device memory (for example a host program with no device
+ * allocator of its own, or a process that fixes its memory budget at
+ * start-up).  The paper has no counterpart: this is a deployment variant of
+ * poetx_cnp_build with the same arguments (minus ws) and the same result.
+ * Scratch is a 24 MiB device array inside the library, held by every GPU
+ * that loads it until the process exits; it fits Q, S and H of up to
+ * nblk*b*b ~= 2.09e6 fp32 elements (b = 256: nblk <= 31; b = 512: nblk <= 7).
+ * Larger requests return POETX_E_WORKSPACE without queueing anything.  The
+ * first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  All calls share the one array and its contents
+ * persist between calls (nothing in it needs to start at zero): calls whose
+ * work overlaps on the GPU (other streams, other threads) race on it, so
+ * order them on one stream or synchronise between them. */
+poetx_status poetx_cnp_build_fixed(int32_t nblk, int32_t b, const float* q, int32_t dtype, void* G, void* stream);
+
 /* Backward of poetx_cnp_build: given dG = dL/dG [nblk][b][b] (fp32), writes
  * dq = dL/dq [nblk][b(b-1)/2] (fp32), dq_k = dL/dQ[i][j] - dL/dQ[j][i].
  * accumulate != 0 adds to dq instead of overwriting it.  dtype names the

@@ -54,6 +54,7 @@ SIGNATURES = {
     "poetx_frame_export": (ctypes.c_int, [_LP, _VP, _VP]),
     "poetx_cnp_build": (ctypes.c_int, [_I32, _I32, _VP, _I32, _VP, _VP, _SZ, _VP]),
     "poetx_cnp_backward": (ctypes.c_int, [_I32, _I32, _VP, _VP, _VP, _I32, _I32, _VP, _SZ, _VP]),
+    "poetx_cnp_build_fixed": (ctypes.c_int, [_I32, _I32, _VP, _I32, _VP, _VP]),
     "poetx_layer_cnp_workspace_bytes": (_SZ, [_LP]),
     "poetx_layer_cnp_build": (ctypes.c_int, [_LP, _VP, _SZ, _VP]),
     "poetx_forward": (ctypes.c_int, [_LP, _I64, _VP, _VP, _VP, _VP, _SZ, _VP]),
@@ -156,6 +157,11 @@ def poetx_frame_export(layer: poetx_layer, W0lin, stream=None) -> None:
 def poetx_cnp_build(nblk: int, b: int, q, dtype: int, G, ws, ws_bytes: int, stream=None) -> None:
     _check(lib().poetx_cnp_build(nblk, b, _ptr(q), dtype, _ptr(G), _ptr(ws), ws_bytes, _stream(stream)),
            "poetx_cnp_build")
+
+
+def poetx_cnp_build_fixed(nblk: int, b: int, q, dtype: int, G, stream=None) -> None:
+    """poetx_cnp_build with the library's fixed device scratch (no workspace)."""
+    _check(lib().poetx_cnp_build_fixed(nblk, b, _ptr(q), dtype, _ptr(G), _stream(stream)), "poetx_cnp_build_fixed")
 
 
 def poetx_cnp_backward(nblk: int, b: int, q, dG, dq, accumulate: int, dtype: int, ws, ws_bytes: int,

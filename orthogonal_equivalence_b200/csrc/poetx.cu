@@ -1039,3 +1039,55 @@ poetx_status poetx_profile_end(double* ms_per_stage, int64_t* launches_per_stage
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- fixed-scratch CNP build
+// Some callers cannot allocate device memory when they build G: a host
+// program that links only this C library and has no device allocator of its
+// own, or a serving process that reserves its whole memory budget at start-up
+// and forbids allocations afterwards.  For them poetx_cnp_build_fixed takes
+// its scratch (Q, S and H for every block) from this file-scope device array
+// instead of a caller workspace.  The array is kFixedScratchBytes on every
+// GPU that loads the library, for the life of the process.  Host code must
+// not hand the symbol itself to a kernel (on the host it only names the
+// array); the device address comes from cudaGetSymbolAddress, looked up once
+// per device on that device's first call.
+constexpr size_t kFixedScratchBytes = size_t(24) << 20;
+static __device__ __align__(256) unsigned char g_cnp_fixed_scratch[kFixedScratchBytes];
+
+namespace {
+std::mutex g_fixed_mu;
+void* g_fixed_scratch_ptr[64] = {nullptr};
+
+// Device address of the fixed scratch on the current device `dev`.
+poetx_status fixed_scratch(int dev, void** out) {
+  std::lock_guard<std::mutex> g(g_fixed_mu);
+  if (!g_fixed_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_cnp_fixed_scratch) != cudaSuccess || !p) {
+      (void)cudaGetLastError();
+      return POETX_E_CUDA;
+    }
+    g_fixed_scratch_ptr[dev] = p;
+  }
+  *out = g_fixed_scratch_ptr[dev];
+  return POETX_OK;
+}
+}  // namespace
+
+extern "C" poetx_status poetx_cnp_build_fixed(int32_t nblk, int32_t b, const float* q, int32_t dtype, void* G,
+                                              void* stream) {
+  POETX_TRY(check_dtype_b(dtype, b));
+  if (nblk < 0) return POETX_E_ARG;
+  if (nblk == 0) return POETX_OK;
+  POETX_TRY(check_ptr(q));
+  POETX_TRY(check_ptr(G));
+  const size_t need = kAlign + 3 * cnp_units(nblk, b);
+  if (need > kFixedScratchBytes) return POETX_E_WORKSPACE;  // too many blocks for the fixed scratch
+  int dev;
+  POETX_TRY(current_device(&dev));
+  void* scratch = nullptr;
+  POETX_TRY(fixed_scratch(dev, &scratch));
+  // Q, S and H are written in full before they are read: nothing to clear.
+  Carver c(scratch, kFixedScratchBytes);
+  return cnp_build2(b, dtype, q, nblk, G, nullptr, 0, nullptr, c, static_cast<cudaStream_t>(stream), dev);
+}
