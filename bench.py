@@ -35,9 +35,11 @@ import poetx_inputs as pi  # noqa: E402
 
 METRIC = "POET-X layer fwd+bwd tokens/s (Llama-8B shapes, b=256); % bf16 tensor peak"
 WORKLOAD = "block8b"
-# DRAM bytes per launch of the dominant kernel (w0_gemm) from an ncu capture;
-# None until a capture of the current kernel exists.
-W0_GEMM_TRAFFIC_BYTES = None
+# DRAM bytes (read + write) per launch of the dominant kernel -- the forward
+# W0 GEMM at M = 16384, N = 14336, K = 4096 -- from an ncu capture of that
+# kernel and shape (dram__bytes_read.sum + dram__bytes_write.sum); reset to
+# None whenever the kernel changes until it is captured again.
+W0_GEMM_TRAFFIC_BYTES = 1073310208 + 453245440
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -245,6 +247,7 @@ def bench_poetx(args, cfg: pi.Config) -> dict:
     end.record(stream)
     torch.cuda.synchronize(device)
     stages = px.poetx_profile_end()
+    records = px.poetx_profile_records()
     barrier(device)
     clocks = sampler.stop()
     ms_local = start.elapsed_time(end)
@@ -286,7 +289,18 @@ def bench_poetx(args, cfg: pi.Config) -> dict:
     w0_ms, w0_launches = stages["w0_gemm"]
     w0_flops = cfg.gemm_flops_per_step() * args.steps  # 2Tmn forward + 2Tmn backward per linear
     peak_sus = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
-    achieved = w0_flops / (w0_ms / 1e3) / 1e12 if w0_ms > 0 else None
+    # Dominant kernel: the forward W0 GEMM (Y = U W~, M = T, N = n, K = m) of
+    # the linears with the largest m x n and that exact shape (gate and up in
+    # the 8B block).  W0 launches per step: forward in layer order, then
+    # backward in reverse order.
+    L = len(cfg.layers)
+    big = max(m * n for _, m, n in cfg.layers)
+    shape = next((m, n) for _, m, n in cfg.layers if m * n == big)
+    dom_layers = [i for i, (_, m, n) in enumerate(cfg.layers) if (m, n) == shape]
+    w0_rec = [ms for st, ms in records if st == "w0_gemm"]
+    dom_ms = [ms for k, ms in enumerate(w0_rec) if (k % (2 * L)) < L and (k % (2 * L)) in dom_layers]
+    dom_flops = 2.0 * cfg.T * shape[0] * shape[1]
+    achieved = dom_flops / (statistics.mean(dom_ms) / 1e3) / 1e12 if dom_ms else None
     total_launches = int(sum(c for _, c in stages.values()))
     res = {
         "metric": METRIC,
@@ -304,15 +318,20 @@ def bench_poetx(args, cfg: pi.Config) -> dict:
         "config": config_block(cfg, world),
         "tflops_per_gpu": flops_step / (ms_step / 1e3) / 1e12,
         "pct_bf16_peak": 100.0 * flops_step / (ms_step / 1e3) / 1e12 / peak_sus,
-        "roofline": {"kernel": "w0_gemm", "bound": "tensor", "achieved": achieved,
+        "roofline": {"kernel": f"w0_gemm forward, M={cfg.T} N={shape[1]} K={shape[0]} "
+                               f"(layers {[cfg.layers[i][0] for i in dom_layers]})",
+                     "bound": "tensor", "achieved": achieved,
                      "peak": peak_sus, "unit": "TFLOP/s",
                      "frac": (achieved / peak_sus) if achieved else None,
-                     "traffic": W0_GEMM_TRAFFIC_BYTES,
+                     "traffic": W0_GEMM_TRAFFIC_BYTES if (cfg.name, cfg.T) == ("block8b", 16384) else None,
                      "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)",
-                     "launches": w0_launches,
-                     "algorithmic_flops_per_launch": 2 * sum(cfg.T * m * n for _, m, n in cfg.layers) / len(cfg.layers),
-                     "note": "achieved = algorithmic 2*T*m*n per launch / mean CUDA-event launch time, "
-                             "forward (Y = U W~) and backward (dU = dY W~^T) launches of all 7 linears"},
+                     "launches": len(dom_ms),
+                     "algorithmic_flops_per_launch": dom_flops,
+                     "algorithmic_bytes_per_launch": 2.0 * (cfg.T * shape[0] + shape[0] * shape[1] + cfg.T * shape[1]),
+                     "note": "achieved = 2*T*m*n per launch / mean CUDA-event launch time over the timed region; "
+                             "traffic = DRAM bytes per launch of the same kernel and shape from an ncu capture"},
+        "w0_stage": {"tflops": w0_flops / (w0_ms / 1e3) / 1e12 if w0_ms > 0 else None, "launches": w0_launches,
+                     "note": "all forward and backward W0 GEMM launches of the step"},
         "stages_ms_per_step": {k: v[0] / args.steps for k, v in stages.items()},
         "gpu_launches": total_launches,
         "clocks": clocks,
@@ -396,6 +415,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["poetx", "reference"], default="poetx")
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(pi.CONFIGS))
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override the workload's tokens per GPU (smaller cases for profiler captures)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-tokens", type=int, default=512, help="token sample of the CPU-baseline leg")
@@ -404,6 +425,9 @@ def main(argv=None):
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     cfg = pi.CONFIGS[args.workload]
+    if args.tokens is not None:
+        import dataclasses
+        cfg = dataclasses.replace(cfg, T=args.tokens)
     res = bench_reference(args, cfg) if args.impl == "reference" else bench_poetx(args, cfg)
     if res is not None:
         print(json.dumps(res), flush=True)

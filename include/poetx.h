@@ -184,6 +184,10 @@ int32_t poetx_profile_stage_count(void);
 const char* poetx_profile_stage_name(int32_t stage);
 poetx_status poetx_profile_begin(void);
 poetx_status poetx_profile_end(double* ms_per_stage, int64_t* launches_per_stage, int32_t nstages);
+/* Per-launch records of the last finished profiling session, in launch
+ * order: stage index and device ms (HOST arrays of max_records entries).
+ * Returns the number of records (pass NULL / 0 to query it). */
+int32_t poetx_profile_records(int32_t* stages, float* ms, int32_t max_records);
 
 #ifdef __cplusplus
 }

@@ -65,6 +65,7 @@ SIGNATURES = {
     "poetx_profile_stage_name": (ctypes.c_char_p, [_I32]),
     "poetx_profile_begin": (ctypes.c_int, []),
     "poetx_profile_end": (ctypes.c_int, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64), _I32]),
+    "poetx_profile_records": (_I32, [ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_float), _I32]),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -211,6 +212,16 @@ def poetx_profile_end() -> dict:
     cnt = (ctypes.c_int64 * n)()
     _check(lib().poetx_profile_end(ms, cnt, n), "poetx_profile_end")
     return {lib().poetx_profile_stage_name(i).decode(): (ms[i], cnt[i]) for i in range(n)}
+
+
+def poetx_profile_records() -> list:
+    """[(stage name, device ms)] per launch of the last profiling session."""
+    n = lib().poetx_profile_records(None, None, 0)
+    st = (ctypes.c_int32 * max(n, 1))()
+    ms = (ctypes.c_float * max(n, 1))()
+    lib().poetx_profile_records(st, ms, n)
+    names = [lib().poetx_profile_stage_name(i).decode() for i in range(lib().poetx_profile_stage_count())]
+    return [(names[st[i]], ms[i]) for i in range(n)]
 
 
 from .layer import PoetxLinear  # noqa: E402,F401

@@ -126,6 +126,7 @@ struct Profiler {
   std::vector<cudaEvent_t> pool;
   size_t used = 0;
   std::vector<std::pair<int, size_t>> recs;  // (stage, index of the start event)
+  std::vector<std::pair<int, float>> done;   // (stage, ms) of the last finished session
 };
 
 Profiler& profiler() {
@@ -1003,6 +1004,7 @@ poetx_status poetx_profile_begin(void) {
   P.on = true;
   P.used = 0;
   P.recs.clear();
+  P.done.clear();
   return POETX_OK;
 }
 
@@ -1031,11 +1033,25 @@ poetx_status poetx_profile_end(double* ms_per_stage, int64_t* launches_per_stage
       ms_per_stage[r.first] += ms;
       launches_per_stage[r.first] += 1;
     }
+    P.done.emplace_back(r.first, ms);
   }
   P.on = false;
   P.used = 0;
   P.recs.clear();
   return st;
+}
+
+int32_t poetx_profile_records(int32_t* stages, float* ms, int32_t max_records) {
+  Profiler& P = profiler();
+  std::lock_guard<std::mutex> g(P.mu);
+  const int32_t n = static_cast<int32_t>(P.done.size());
+  if (!stages || !ms || max_records <= 0) return n;
+  const int32_t k = n < max_records ? n : max_records;
+  for (int32_t i = 0; i < k; ++i) {
+    stages[i] = P.done[i].first;
+    ms[i] = P.done[i].second;
+  }
+  return n;
 }
 
 }  // extern "C"

@@ -1,0 +1,83 @@
+"""CPU checks of bench.py: the data-parallel plumbing (gradient all-reduce,
+max-over-ranks timing, barrier) on two gloo ranks, and the JSON contract of
+the oracle arm (--impl reference) on a small workload."""
+import datetime
+import json
+import multiprocessing as mp
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    import bench
+    flat = torch.full((17,), float(rank + 1))
+    bench.allreduce_grads(flat)
+    slowest = bench.reduce_max(10.0 * rank + 1.5, torch.device("cpu"))
+    bench.barrier(torch.device("cpu"))
+    out.put((rank, flat.tolist(), slowest))
+    dist.destroy_process_group()
+
+
+def test_two_rank_gradient_allreduce_and_max_timing():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, flat, slowest in res:
+        assert flat == [3.0] * 17          # sum of 1 and 2 on every rank
+        assert slowest == 11.5            # max over ranks of the per-rank times
+
+
+def test_reference_arm_json_contract():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
+                          "tiny", "--steps", "2", "--warmup", "3", "--ref-tokens", "16"],
+                         capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr
+    line = json.loads(out.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference"
+    assert line["unit"] == "tokens/s" and line["value"] > 0 and line["higher_is_better"] is True
+    assert line["steps"] == 2 and line["warmup"] == 3
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
+
+
+def test_reference_arm_other_ranks_do_no_work(monkeypatch):
+    sys.path.insert(0, ROOT)
+    import bench
+    import poetx_inputs as pi
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+
+    class A:
+        ref_tokens, warmup, steps = 4, 3, 1
+
+    assert bench.bench_reference(A, pi.CONFIGS["tiny"]) is None
+
+
+def test_bench_rejects_short_warmup():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--warmup", "2"],
+                         capture_output=True, text=True, timeout=120, cwd=ROOT)
+    assert out.returncode != 0
