@@ -253,7 +253,11 @@ def bench_poetx(args, cfg: pi.Config) -> dict:
     ms_local = start.elapsed_time(end)
     ms_total = reduce_max(ms_local, device)
 
-    # end to end through the public API: pinned host inputs in, gradients out
+    # End to end through the public API: every step copies its inputs (x and
+    # dz of every linear) from pinned host memory and reads the packed
+    # gradients back.  The copies run on their own stream into two alternating
+    # sets of device buffers, so step s+1's inputs stream in while step s
+    # computes; each linear waits only for its own inputs.
     e2e = None
     if not args.no_e2e:
         host_x = [l["x"].cpu().pin_memory() for l in layers]
@@ -261,26 +265,53 @@ def bench_poetx(args, cfg: pi.Config) -> dict:
         host_dq = torch.empty(flat.numel(), dtype=torch.float32).pin_memory()
         h2d = sum(t.numel() * t.element_size() for t in host_x + host_dz)
         d2h = host_dq.numel() * 4
-        e_steps = max(1, min(args.steps, 5))
+        e_steps = max(2, min(args.steps, 6))
+        copy_stream = torch.cuda.Stream(device)
+        dev_x = [[l["x"] for l in layers], [torch.empty_like(l["x"]) for l in layers]]
+        dev_dz = [[l["dz"] for l in layers], [torch.empty_like(l["dz"]) for l in layers]]
+        ev = lambda: torch.cuda.Event()  # noqa: E731
+        x_ready = [[ev() for _ in layers] for _ in range(2)]
+        dz_ready = [[ev() for _ in layers] for _ in range(2)]
+        consumed = [[ev() for _ in layers] for _ in range(2)]
+        for k in range(2):
+            for e in consumed[k]:
+                e.record(stream)
 
-        def e2e_step():
-            for l, hx, hdz in zip(layers, host_x, host_dz):
-                l["x"].copy_(hx, non_blocking=True)
-                l["dz"].copy_(hdz, non_blocking=True)
-            run_step(layers, flat)
+        def e2e_step(k):
+            with torch.cuda.stream(copy_stream):
+                for i, l in enumerate(layers):
+                    copy_stream.wait_event(consumed[k][i])
+                    dev_x[k][i].copy_(host_x[i], non_blocking=True)
+                    x_ready[k][i].record(copy_stream)
+                for i in reversed(range(len(layers))):
+                    dev_dz[k][i].copy_(host_dz[i], non_blocking=True)
+                    dz_ready[k][i].record(copy_stream)
+            for i, l in enumerate(layers):
+                stream.wait_event(x_ready[k][i])
+                l["L"].build()
+                l["L"].forward(dev_x[k][i], z=l["z"], y=l["y"])
+            for i in reversed(range(len(layers))):
+                l = layers[i]
+                stream.wait_event(dz_ready[k][i])
+                l["L"].backward(dev_x[k][i], l["y"], dev_dz[k][i], dx=l["dx"], dqR=l["dqR"], dqP=l["dqP"])
+                consumed[k][i].record(stream)
+            allreduce_grads(flat)
             host_dq.copy_(flat, non_blocking=True)
 
-        e2e_step()
+        e2e_step(0)
+        e2e_step(1)
         barrier(device)
         s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s2.record(stream)
-        for _ in range(e_steps):
-            e2e_step()
+        copy_stream.wait_event(s2)
+        for it in range(e_steps):
+            e2e_step(it % 2)
         e2.record(stream)
         torch.cuda.synchronize(device)
         e_ms = reduce_max(s2.elapsed_time(e2), device)
         e2e = {"value": world * cfg.T * e_steps / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "steps": e_steps}
+               "d2h_bytes_per_step": d2h, "steps": e_steps,
+               "h2d_gbs": h2d * e_steps / (e_ms / 1e3) / 1e9}
     device_error = px.poetx_device_error()
 
     peaks, peak_src = measured_peaks()

@@ -18,77 +18,6 @@ __device__ __forceinline__ int64_t tri_index(int64_t i, int64_t j, int64_t b) {
   return i * (b - 1) - i * (i - 1) / 2 + (j - i - 1);
 }
 
-// One warp per row of the triangle: lanes read the row's contiguous run of
-// q and write Q[i][j] = q (coalesced) and Q[j][i] = -q; lane 0 writes the
-// zero diagonal entry.  grid.x covers nblk*b rows, 8 warps per block.
-__global__ void unpack_skew_kernel(const float* __restrict__ q, int nblk, int b, float* __restrict__ Q) {
-  const int64_t row_global = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row_global >= static_cast<int64_t>(nblk) * b) return;
-  const int64_t blk = row_global / b;
-  const int i = static_cast<int>(row_global - blk * b);
-  const int64_t L = static_cast<int64_t>(b) * (b - 1) / 2;
-  const float* qb = q + blk * L;
-  float* Qb = Q + blk * b * b;
-  const int64_t k0 = tri_index(i, i + 1, b);
-  for (int j = i + 1 + lane; j < b; j += 32) {
-    const float v = qb[k0 + (j - i - 1)];
-    Qb[static_cast<int64_t>(i) * b + j] = v;
-    Qb[static_cast<int64_t>(j) * b + i] = -v;
-  }
-  if (lane == 0) Qb[static_cast<int64_t>(i) * b + i] = 0.f;
-}
-
-// out = a*X + c*Y (fp32, n elements)
-__global__ void axpby_kernel(const float* __restrict__ X, float a, const float* __restrict__ Y, float c,
-                             float* __restrict__ out, int64_t n) {
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
-    out[i] = a * X[i] + c * Y[i];
-}
-
-// dq[k(i,j)] (+)= dA[i][j] - dA[j][i]; one block row per (blk, i).
-__global__ void fold_skew_kernel(const float* __restrict__ dA, int nblk, int b, float* __restrict__ dq,
-                                 int accumulate) {
-  const int64_t row_global = blockIdx.x;
-  const int64_t blk = row_global / b;
-  const int i = static_cast<int>(row_global - blk * b);
-  const int64_t L = static_cast<int64_t>(b) * (b - 1) / 2;
-  const float* Ab = dA + blk * b * b;
-  float* qb = dq + blk * L;
-  const int64_t k0 = tri_index(i, i + 1, b);
-  for (int j = i + 1 + threadIdx.x; j < b; j += blockDim.x) {
-    const float g = Ab[static_cast<int64_t>(i) * b + j] - Ab[static_cast<int64_t>(j) * b + i];
-    const int64_t k = k0 + (j - i - 1);
-    qb[k] = accumulate ? qb[k] + g : g;
-  }
-}
-
-// out[e] = sum_{s < splits} part[s*count + e], summed in split order (the
-// result does not depend on the launch shape).
-__global__ void reduce_splits_kernel(const float* __restrict__ part, int splits, int64_t count,
-                                     float* __restrict__ out) {
-  const int64_t n4 = count / 4;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    float4 acc = reinterpret_cast<const float4*>(part)[i];
-    for (int s = 1; s < splits; ++s) {
-      const float4 v = reinterpret_cast<const float4*>(part + s * count)[i];
-      acc.x += v.x;
-      acc.y += v.y;
-      acc.z += v.z;
-      acc.w += v.w;
-    }
-    reinterpret_cast<float4*>(out)[i] = acc;
-  }
-  for (int64_t i = n4 * 4 + static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < count;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    float acc = part[i];
-    for (int s = 1; s < splits; ++s) acc += part[s * count + i];
-    out[i] = acc;
-  }
-}
-
 // G blocks := I (the state right after a merge), in the layer's dtype.
 template <typename T>
 __global__ void identity_blocks_kernel(T* __restrict__ G, int nblk, int b) {
@@ -133,33 +62,43 @@ __global__ void transpose_blocks_kernel(const T* __restrict__ in, float* __restr
 // Matrices live in row-strided block arrays: block t starts at t * bs, rows
 // ld apart (so a block can sit inside a wider concatenated row).
 
-// Unpack packed triangles into Q (and optionally a second copy); one warp
-// per triangle row.  grid.x covers nblk * b rows, 8 warps per block.
+// Unpack packed triangles into Q (and optionally a second copy).  One block
+// per 32 x 32 tile (ti, tj) with ti <= tj of one b x b block: row i of the
+// tile reads its run of q (contiguous for i < j), writes Q[i][j] = q and,
+// through a shared-memory transpose, the mirrored tile Q[j][i] = -q, so both
+// the reads and the writes are coalesced.  grid (b/32, b/32, nblk), block
+// (32, 8); tiles below the diagonal exit at once.
 __global__ void unpack_skew2_kernel(const float* __restrict__ q0, int n0, const float* __restrict__ q1, int nblk,
                                     int b, float* __restrict__ o1, int64_t ld1, int64_t bs1, float* __restrict__ o2,
                                     int64_t ld2, int64_t bs2) {
-  const int64_t row_global = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row_global >= static_cast<int64_t>(nblk) * b) return;
-  const int blk = static_cast<int>(row_global / b);
-  const int i = static_cast<int>(row_global - static_cast<int64_t>(blk) * b);
+  __shared__ float tile[32][33];
+  const int ti = blockIdx.y, tj = blockIdx.x, blk = blockIdx.z;
+  if (ti > tj || blk >= nblk) return;
   const int64_t L = static_cast<int64_t>(b) * (b - 1) / 2;
   const float* qb = blk < n0 ? q0 + blk * L : q1 + (blk - n0) * L;
   float* A1 = o1 + blk * bs1;
   float* A2 = o2 ? o2 + blk * bs2 : nullptr;
-  const int64_t k0 = tri_index(i, i + 1, b);
-  for (int j = i + 1 + lane; j < b; j += 32) {
-    const float v = qb[k0 + (j - i - 1)];
-    A1[i * ld1 + j] = v;
-    A1[j * ld1 + i] = -v;
-    if (A2) {
-      A2[i * ld2 + j] = v;
-      A2[j * ld2 + i] = -v;
+  const int r0 = ti * 32, c0 = tj * 32;
+  for (int ii = threadIdx.y; ii < 32; ii += 8) {
+    const int i = r0 + ii, j = c0 + threadIdx.x;
+    float v = 0.f;
+    if (i < b && j < b) {
+      if (i < j) v = qb[tri_index(i, j, b)];
+      else if (i > j) v = -qb[tri_index(j, i, b)];  // diagonal tile, lower half
+      A1[i * ld1 + j] = v;
+      if (A2) A2[i * ld2 + j] = v;
     }
+    tile[ii][threadIdx.x] = v;
   }
-  if (lane == 0) {
-    A1[i * ld1 + i] = 0.f;
-    if (A2) A2[i * ld2 + i] = 0.f;
+  if (ti == tj) return;  // a diagonal tile is its own mirror
+  __syncthreads();
+  for (int jj = threadIdx.y; jj < 32; jj += 8) {
+    const int j = c0 + jj, i = r0 + threadIdx.x;
+    if (i < b && j < b) {
+      const float v = -tile[threadIdx.x][jj];
+      A1[j * ld1 + i] = v;
+      if (A2) A2[j * ld2 + i] = v;
+    }
   }
 }
 

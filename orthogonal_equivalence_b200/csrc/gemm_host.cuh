@@ -169,7 +169,14 @@ cudaError_t launch_tc_bn(const GemmDesc& g, cudaStream_t st, int device) {
 
 inline cudaError_t launch_tc(const GemmDesc& g, cudaStream_t st, int device) {
   const bool tf32 = g.A.et == ET_F32;
-  switch (choose_bn(g.N)) {
+  int bn = choose_bn(g.N);
+  // Small batched products (the CNP blocks) fill few SMs with 256-wide tiles:
+  // halve the tile width when that leaves more than a quarter of the SMs idle.
+  if (bn == 256) {
+    const int64_t tiles = int64_t(g.batch) * g.splits * ((g.M + tc::BM - 1) / tc::BM) * (g.N / 256);
+    if (4 * tiles < 3 * int64_t(sm_count(device))) bn = 128;
+  }
+  switch (bn) {
     case 256: return tf32 ? launch_tc_bn<256, true>(g, st, device) : launch_tc_bn<256, false>(g, st, device);
     case 128: return tf32 ? launch_tc_bn<128, true>(g, st, device) : launch_tc_bn<128, false>(g, st, device);
     default: return tf32 ? launch_tc_bn<64, true>(g, st, device) : launch_tc_bn<64, false>(g, st, device);

@@ -499,9 +499,9 @@ poetx_status cnp_build2(int32_t b, int32_t dtype, const float* q0, int n0, void*
   float* H = ws.take<float>(sizeof(float) * nbb);
   const bool tc_path = use_tc(dtype);
   const int64_t bb = int64_t(b) * b;
+  const dim3 ugrid((b + 31) / 32, (b + 31) / 32, nblk), ublock(32, 8);
   PROFILED(ST_CNP_ELEM, st,
-           unpack_skew2_kernel<<<static_cast<int>((int64_t(nblk) * b + 7) / 8), 256, 0, st>>>(
-               q0, n0, q1, nblk, b, Q, b, bb, nullptr, 0, 0));
+           unpack_skew2_kernel<<<ugrid, ublock, 0, st>>>(q0, n0, q1, nblk, b, Q, b, bb, nullptr, 0, 0));
   POETX_CUDA(cudaGetLastError());
   // S = -(Q Q^T); H = S + 2Q as a second output
   {
@@ -552,9 +552,9 @@ poetx_status cnp_backward2(int32_t b, int32_t dtype, const float* q0, int n0, co
   float* dA = ws.take<float>(sizeof(float) * nbb);
   const bool tc_path = use_tc(dtype);
   // A -> X2[:, b:2b] and Y2[:, 0:b]
+  const dim3 ugrid((b + 31) / 32, (b + 31) / 32, nblk), ublock(32, 8);
   PROFILED(ST_CNP_ELEM, st,
-           unpack_skew2_kernel<<<static_cast<int>((int64_t(nblk) * b + 7) / 8), 256, 0, st>>>(
-               q0, n0, q1, nblk, b, X2 + b, b3, b * b3, Y2, b3, b * b3));
+           unpack_skew2_kernel<<<ugrid, ublock, 0, st>>>(q0, n0, q1, nblk, b, X2 + b, b3, b * b3, Y2, b3, b * b3));
   // dG -> X1[:, b:2b], X2[:, 2b:3b];  dG^T -> Y1[:, 0:b]
   {
     const dim3 grid((b + 31) / 32, (b + 31) / 32, nblk), block(32, 8);
