@@ -188,6 +188,7 @@ def build_block(cfg: pi.Config, device, rank: int):
         L = l["L"]
         l["z"] = torch.empty((cfg.T, l["n"]), dtype=torch.bfloat16, device=device)
         l["y"] = torch.empty((cfg.T, l["n"]), dtype=torch.bfloat16, device=device)
+        l["xg"] = torch.empty((cfg.T, l["m"]), dtype=torch.bfloat16, device=device)
         l["dx"] = torch.empty((cfg.T, l["m"]), dtype=torch.bfloat16, device=device)
         l["dqR"] = flat[off:off + L.qR.numel()].view_as(L.qR)
         off += L.qR.numel()
@@ -197,13 +198,14 @@ def build_block(cfg: pi.Config, device, rank: int):
 
 
 def run_step(layers, flat) -> None:
+    # the forward keeps Y and Xg = x[:, permR] for the backward ("fast" variant)
     for l in layers:
         L = l["L"]
         L.build()
-        L.forward(l["x"], z=l["z"], y=l["y"])
+        l["saved"] = L.forward(l["x"], save_xg=True, z=l["z"], y=l["y"], xg=l["xg"])[1]
     for l in reversed(layers):
         L = l["L"]
-        L.backward(l["x"], l["y"], l["dz"], dx=l["dx"], dqR=l["dqR"], dqP=l["dqP"])
+        L.backward(l["x"], l["saved"], l["dz"], dx=l["dx"], dqR=l["dqR"], dqP=l["dqP"])
     allreduce_grads(flat)
 
 
@@ -289,11 +291,11 @@ def bench_poetx(args, cfg: pi.Config) -> dict:
             for i, l in enumerate(layers):
                 stream.wait_event(x_ready[k][i])
                 l["L"].build()
-                l["L"].forward(dev_x[k][i], z=l["z"], y=l["y"])
+                l["saved"] = l["L"].forward(dev_x[k][i], save_xg=True, z=l["z"], y=l["y"], xg=l["xg"])[1]
             for i in reversed(range(len(layers))):
                 l = layers[i]
                 stream.wait_event(dz_ready[k][i])
-                l["L"].backward(dev_x[k][i], l["y"], dev_dz[k][i], dx=l["dx"], dqR=l["dqR"], dqP=l["dqP"])
+                l["L"].backward(dev_x[k][i], l["saved"], dev_dz[k][i], dx=l["dx"], dqR=l["dqR"], dqP=l["dqP"])
                 consumed[k][i].record(stream)
             allreduce_grads(flat)
             host_dq.copy_(flat, non_blocking=True)

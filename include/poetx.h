@@ -143,19 +143,21 @@ poetx_status poetx_cnp_backward(int32_t nblk, int32_t b, const float* q, const f
 /* Forward (section 1, input-centric): z = x R W0 P for T token rows.
  * x [T][m], z [T][n] in natural feature order (dtype).  y_save [T][n] (dtype)
  * receives Y = (x Psi_R^T Diag(G_R)) W (the P-side input, in the Psi_P
- * frame) for the backward; pass NULL for inference.  Uses layer->GR/GP as
- * last built by poetx_cnp_build.  T = 0 is a no-op. */
-poetx_status poetx_forward(const poetx_layer* layer, int64_t T, const void* x, void* z, void* y_save, void* ws,
-                           size_t ws_bytes, void* stream);
+ * frame) for the backward; pass NULL for inference.  xg_save [T][m] (dtype,
+ * nullable) receives Xg = x Psi_R^T, which spares the backward a gather of x.
+ * Uses layer->GR/GP as last built by poetx_cnp_build.  T = 0 is a no-op. */
+poetx_status poetx_forward(const poetx_layer* layer, int64_t T, const void* x, void* z, void* y_save,
+                           void* xg_save, void* ws, size_t ws_bytes, void* stream);
 
 /* Backward of L = <dz, z>: dx [T][m] (dtype; NULL skips it) and the packed
  * gradients dqR [m/b][b(b-1)/2], dqP [n/b][b(b-1)/2] (fp32; overwritten, or
- * added to when accumulate != 0).  Needs x and the y_save of the matching
- * forward; W0 is frozen, so no dW0.  The dq sums over tokens use a fixed
- * split and order (deterministic for a given shape). */
+ * added to when accumulate != 0).  Needs the y_save of the matching forward
+ * and either its xg_save or (xg_save == NULL) the input x, which is then
+ * gathered again; W0 is frozen, so no dW0.  The dq sums over tokens use a
+ * fixed split and order (deterministic for a given shape). */
 poetx_status poetx_backward(const poetx_layer* layer, int64_t T, const void* x, const void* y_save,
-                            const void* dz, void* dx, float* dqR, float* dqP, int32_t accumulate, void* ws,
-                            size_t ws_bytes, void* stream);
+                            const void* xg_save, const void* dz, void* dx, float* dqR, float* dqP,
+                            int32_t accumulate, void* ws, size_t ws_bytes, void* stream);
 
 /* Merge (merge_if_needed in the write-up's API snippet): writes into W_out
  * ([n][m], dtype, must not overlap layer->W) the weight R W0 P expressed in

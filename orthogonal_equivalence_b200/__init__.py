@@ -57,8 +57,8 @@ SIGNATURES = {
     "poetx_cnp_build_fixed": (ctypes.c_int, [_I32, _I32, _VP, _I32, _VP, _VP]),
     "poetx_layer_cnp_workspace_bytes": (_SZ, [_LP]),
     "poetx_layer_cnp_build": (ctypes.c_int, [_LP, _VP, _SZ, _VP]),
-    "poetx_forward": (ctypes.c_int, [_LP, _I64, _VP, _VP, _VP, _VP, _SZ, _VP]),
-    "poetx_backward": (ctypes.c_int, [_LP, _I64, _VP, _VP, _VP, _VP, _VP, _VP, _I32, _VP, _SZ, _VP]),
+    "poetx_forward": (ctypes.c_int, [_LP, _I64, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "poetx_backward": (ctypes.c_int, [_LP, _I64, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I32, _VP, _SZ, _VP]),
     "poetx_merge": (ctypes.c_int, [_LP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "poetx_check_perm": (ctypes.c_int, [_VP, _I32, _VP, _VP, _SZ, _VP]),
     "poetx_profile_stage_count": (_I32, []),
@@ -180,15 +180,16 @@ def poetx_layer_cnp_build(layer: poetx_layer, ws, ws_bytes: int, stream=None) ->
            "poetx_layer_cnp_build")
 
 
-def poetx_forward(layer: poetx_layer, T: int, x, z, y_save, ws, ws_bytes: int, stream=None) -> None:
-    _check(lib().poetx_forward(ctypes.byref(layer), T, _ptr(x), _ptr(z), _ptr(y_save), _ptr(ws), ws_bytes,
-                               _stream(stream)), "poetx_forward")
+def poetx_forward(layer: poetx_layer, T: int, x, z, y_save, xg_save, ws, ws_bytes: int, stream=None) -> None:
+    _check(lib().poetx_forward(ctypes.byref(layer), T, _ptr(x), _ptr(z), _ptr(y_save), _ptr(xg_save), _ptr(ws),
+                               ws_bytes, _stream(stream)), "poetx_forward")
 
 
-def poetx_backward(layer: poetx_layer, T: int, x, y_save, dz, dx, dqR, dqP, accumulate: int, ws, ws_bytes: int,
-                   stream=None) -> None:
-    _check(lib().poetx_backward(ctypes.byref(layer), T, _ptr(x), _ptr(y_save), _ptr(dz), _ptr(dx), _ptr(dqR),
-                                _ptr(dqP), accumulate, _ptr(ws), ws_bytes, _stream(stream)), "poetx_backward")
+def poetx_backward(layer: poetx_layer, T: int, x, y_save, xg_save, dz, dx, dqR, dqP, accumulate: int, ws,
+                   ws_bytes: int, stream=None) -> None:
+    _check(lib().poetx_backward(ctypes.byref(layer), T, _ptr(x), _ptr(y_save), _ptr(xg_save), _ptr(dz), _ptr(dx),
+                                _ptr(dqR), _ptr(dqP), accumulate, _ptr(ws), ws_bytes, _stream(stream)),
+           "poetx_backward")
 
 
 def poetx_merge(layer: poetx_layer, new_permR, new_permP, W_out, ws, ws_bytes: int, stream=None) -> None:

@@ -727,14 +727,15 @@ poetx_status poetx_cnp_backward(int32_t nblk, int32_t b, const float* q, const f
                        static_cast<cudaStream_t>(stream), dev);
 }
 
-poetx_status poetx_forward(const poetx_layer* layer, int64_t T, const void* x, void* z, void* y_save, void* ws,
-                           size_t ws_bytes, void* stream) {
+poetx_status poetx_forward(const poetx_layer* layer, int64_t T, const void* x, void* z, void* y_save,
+                           void* xg_save, void* ws, size_t ws_bytes, void* stream) {
   POETX_TRY(check_layer(layer));
   if (T < 0) return POETX_E_ARG;
   if (T == 0) return POETX_OK;
   POETX_TRY(check_ptr(x));
   POETX_TRY(check_ptr(z));
   if (y_save && !aligned16(y_save)) return POETX_E_ALIGN;
+  if (xg_save && !aligned16(xg_save)) return POETX_E_ALIGN;
   if (!ws || ws_bytes < fwd_ws(layer, T)) return POETX_E_WORKSPACE;
   int dev;
   POETX_TRY(current_device(&dev));
@@ -744,7 +745,8 @@ poetx_status poetx_forward(const poetx_layer* layer, int64_t T, const void* x, v
   const size_t es = dtype_size(L.dtype);
   const bool tc_path = use_tc(L.dtype);
   Carver c(ws, ws_bytes);
-  void* Xg = c.take<uint8_t>(es * T * L.m);
+  void* Xw = c.take<uint8_t>(es * T * L.m);
+  void* Xg = xg_save ? xg_save : Xw;
   void* U = c.take<uint8_t>(es * T * L.m);
   void* V = c.take<uint8_t>(es * T * L.n);
   void* Yw = c.take<uint8_t>(es * T * L.n);
@@ -783,8 +785,8 @@ poetx_status poetx_forward(const poetx_layer* layer, int64_t T, const void* x, v
 }
 
 poetx_status poetx_backward(const poetx_layer* layer, int64_t T, const void* x, const void* y_save,
-                            const void* dz, void* dx, float* dqR, float* dqP, int32_t accumulate, void* ws,
-                            size_t ws_bytes, void* stream) {
+                            const void* xg_save, const void* dz, void* dx, float* dqR, float* dqP,
+                            int32_t accumulate, void* ws, size_t ws_bytes, void* stream) {
   POETX_TRY(check_layer(layer));
   if (T < 0) return POETX_E_ARG;
   POETX_TRY(check_ptr(dqR));
@@ -800,9 +802,10 @@ poetx_status poetx_backward(const poetx_layer* layer, int64_t T, const void* x, 
     }
     return POETX_OK;
   }
-  POETX_TRY(check_ptr(x));
+  if (!xg_save) POETX_TRY(check_ptr(x));
   POETX_TRY(check_ptr(y_save));
   POETX_TRY(check_ptr(dz));
+  if (xg_save && !aligned16(xg_save)) return POETX_E_ALIGN;
   if (dx && !aligned16(dx)) return POETX_E_ALIGN;
   if (!ws || ws_bytes < bwd_ws(layer, T)) return POETX_E_WORKSPACE;
   int dev;
@@ -850,9 +853,12 @@ poetx_status poetx_backward(const poetx_layer* layer, int64_t T, const void* x, 
     g.C.view_cols = L.m;
     PROFILED(ST_W0, st, POETX_CUDA(launch_gemm(g, tc_path, st, dev)));
   }
-  // Xg = x Psi_R^T (re-gathered; dV is dead)
-  void* Xg = bufA;
-  PROFILED(ST_PERMUTE, st, POETX_CUDA(permute_dt(L.dtype, x, Xg, T, L.m, L.permR, 0, st, dev)));
+  // Xg = x Psi_R^T: the forward's copy when it saved one, else re-gathered (dV is dead)
+  const void* Xg = xg_save;
+  if (!Xg) {
+    Xg = bufA;
+    PROFILED(ST_PERMUTE, st, POETX_CUDA(permute_dt(L.dtype, x, bufA, T, L.m, L.permR, 0, st, dev)));
+  }
   // dXg_j = dU_j G_Rj^T (dY is dead)
   void* dXg = bufB;
   if (dx) PROFILED(ST_BLOCKDIAG, st, POETX_CUDA(launch_gemm(blockdiag_desc(dU, et, T, L.m, L.b, L.GR, true, dXg, et), tc_path, st, dev)));

@@ -8,7 +8,7 @@ triangles qR, qP (the trainable parameters) and the G blocks built from them.
 """
 from __future__ import annotations
 
-from typing import Optional, Tuple
+from typing import NamedTuple, Optional, Tuple
 
 import torch
 
@@ -17,6 +17,13 @@ from . import (POETX_BF16, POETX_FP32, make_layer, poetx_backward, poetx_backwar
                poetx_layer_cnp_build, poetx_layer_cnp_workspace_bytes, poetx_merge, poetx_merge_workspace_bytes)
 
 _TORCH_DTYPE = {POETX_BF16: torch.bfloat16, POETX_FP32: torch.float32}
+
+
+class Saved(NamedTuple):
+    """Activations the forward keeps for the backward: Y ([T][n], the P-side
+    input in the Psi_P frame) and optionally Xg ([T][m], x in the Psi_R frame)."""
+    y: torch.Tensor
+    xg: Optional[torch.Tensor]
 
 
 class PoetxLinear:
@@ -78,23 +85,34 @@ class PoetxLinear:
         poetx_layer_cnp_build(L, ws, nb, stream)
 
     # -------------------------------------------------------------- layer
-    def forward(self, x: torch.Tensor, save: bool = True, z: Optional[torch.Tensor] = None,
-                y: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    def forward(self, x: torch.Tensor, save: bool = True, save_xg: bool = False, z: Optional[torch.Tensor] = None,
+                y: Optional[torch.Tensor] = None, xg: Optional[torch.Tensor] = None,
+                stream=None) -> Tuple[torch.Tensor, Optional["Saved"]]:
+        """z = x R W0 P.  With `save`, also returns what the backward needs:
+        Y (the P-side input) and, with `save_xg`, Xg = x[:, permR]."""
         T = x.shape[0]
         if z is None:
             z = torch.empty((T, self.n), dtype=self.torch_dtype, device=self.device)
         if save and y is None:
             y = torch.empty((T, self.n), dtype=self.torch_dtype, device=self.device)
+        if save and save_xg and xg is None:
+            xg = torch.empty((T, self.m), dtype=self.torch_dtype, device=self.device)
+        if not (save and save_xg):
+            xg = None
         L = self.abi()
         nb = poetx_forward_workspace_bytes(L, T)
         ws = self.workspace("fwd", nb)
-        poetx_forward(L, T, x, z, y if save else None, ws, nb, stream)
-        return z, (y if save else None)
+        poetx_forward(L, T, x, z, y if save else None, xg, ws, nb, stream)
+        return z, (Saved(y, xg) if save else None)
 
-    def backward(self, x: torch.Tensor, y: torch.Tensor, dz: torch.Tensor, need_dx: bool = True,
+    def backward(self, x: torch.Tensor, saved, dz: torch.Tensor, need_dx: bool = True,
                  dx: Optional[torch.Tensor] = None, dqR: Optional[torch.Tensor] = None,
                  dqP: Optional[torch.Tensor] = None, accumulate: bool = False, stream=None):
-        T = x.shape[0]
+        """dx, dqR, dqP of L = <dz, z>.  `saved` is what forward returned (or
+        just the saved Y tensor)."""
+        if isinstance(saved, torch.Tensor):
+            saved = Saved(saved, None)
+        T = dz.shape[0]
         if need_dx and dx is None:
             dx = torch.empty((T, self.m), dtype=self.torch_dtype, device=self.device)
         if dqR is None:
@@ -104,7 +122,8 @@ class PoetxLinear:
         L = self.abi()
         nb = poetx_backward_workspace_bytes(L, T)
         ws = self.workspace("bwd", nb)
-        poetx_backward(L, T, x, y, dz, dx if need_dx else None, dqR, dqP, int(accumulate), ws, nb, stream)
+        poetx_backward(L, T, x, saved.y, saved.xg, dz, dx if need_dx else None, dqR, dqP, int(accumulate), ws, nb,
+                       stream)
         return (dx if need_dx else None), dqR, dqP
 
     def merge(self, new_permR: torch.Tensor, new_permP: torch.Tensor, stream=None) -> None:

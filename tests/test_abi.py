@@ -70,19 +70,21 @@ def test_workspace_sizes_are_host_arithmetic(lib):
 
 def test_validation_before_any_launch(lib):
     # every rejected call returns its status without touching a device
-    assert lib.poetx_forward(None, 10, 4096, 4096, None, 4096, 1 << 30, None) == 1          # E_ARG
+    assert lib.poetx_forward(None, 10, 4096, 4096, None, None, 4096, 1 << 30, None) == 1          # E_ARG
     L = _layer(m=500)
-    assert lib.poetx_forward(ctypes.byref(L), 10, 4096, 4096, None, 4096, 1 << 30, None) == 2  # E_SHAPE
+    assert lib.poetx_forward(ctypes.byref(L), 10, 4096, 4096, None, None, 4096, 1 << 30, None) == 2  # E_SHAPE
     L = _layer(dtype=5)
-    assert lib.poetx_forward(ctypes.byref(L), 10, 4096, 4096, None, 4096, 1 << 30, None) == 3  # E_DTYPE
+    assert lib.poetx_forward(ctypes.byref(L), 10, 4096, 4096, None, None, 4096, 1 << 30, None) == 3  # E_DTYPE
     L = _layer(ptr=4100)
-    assert lib.poetx_forward(ctypes.byref(L), 10, 4096, 4096, None, 4096, 1 << 30, None) == 4  # E_ALIGN
+    assert lib.poetx_forward(ctypes.byref(L), 10, 4096, 4096, None, None, 4096, 1 << 30, None) == 4  # E_ALIGN
     L = _layer()
-    assert lib.poetx_forward(ctypes.byref(L), -1, 4096, 4096, None, 4096, 1 << 30, None) == 1  # T < 0
-    assert lib.poetx_forward(ctypes.byref(L), 10, 4096, 4096, None, 4096, 16, None) == 5       # ws small
-    assert lib.poetx_forward(ctypes.byref(L), 10, None, 4096, None, 4096, 1 << 30, None) == 1  # x NULL
-    assert lib.poetx_backward(ctypes.byref(L), 10, 4096, None, 4096, None, 4096, 4096, 0, 4096, 1 << 30,
+    assert lib.poetx_forward(ctypes.byref(L), -1, 4096, 4096, None, None, 4096, 1 << 30, None) == 1  # T < 0
+    assert lib.poetx_forward(ctypes.byref(L), 10, 4096, 4096, None, None, 4096, 16, None) == 5       # ws small
+    assert lib.poetx_forward(ctypes.byref(L), 10, None, 4096, None, None, 4096, 1 << 30, None) == 1  # x NULL
+    assert lib.poetx_backward(ctypes.byref(L), 10, 4096, None, None, 4096, None, 4096, 4096, 0, 4096, 1 << 30,
                               None) == 1                                                      # y_save NULL
+    assert lib.poetx_backward(ctypes.byref(L), 10, None, 4096, None, 4096, None, 4096, 4096, 0, 4096, 1 << 30,
+                              None) == 1                                                      # no x, no xg
     assert lib.poetx_cnp_build(4, 48, 4096, px.POETX_BF16, 4096, 4096, 1 << 30, None) == 2    # b % 64
     assert lib.poetx_cnp_build(4, 64, 4096, 9, 4096, 4096, 1 << 30, None) == 3
     assert lib.poetx_cnp_build(4, 64, 4096, px.POETX_BF16, 4096, 4096, 8, None) == 5
@@ -100,4 +102,4 @@ def test_no_device_call_fails_cleanly(lib):
     L = _layer()
     T = 10
     ws = px.poetx_forward_workspace_bytes(L, T)
-    assert lib.poetx_forward(ctypes.byref(L), T, 4096, 4096, 4096, 4096, ws, None) == 7
+    assert lib.poetx_forward(ctypes.byref(L), T, 4096, 4096, 4096, None, 4096, ws, None) == 7

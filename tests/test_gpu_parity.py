@@ -194,6 +194,24 @@ def test_empty_and_single_token():
     check(host64(dqR1), dqRo, "bf16", "dqR T=1")
 
 
+@pytest.mark.parametrize("case", [("up8b", 512, 1024, 256, 700), ("tiny", 192, 320, 64, 77)], ids=lambda c: c[0])
+def test_saved_xg_backward_matches_regather(case):
+    # the forward's optional Xg = x[:, permR] gives the backward the same result
+    # (bit for bit) as gathering x again
+    inp = _inputs(*case)
+    L = make_layer(inp)
+    x, dz = dev(inp.x, inp.dtype), dev(inp.dz, inp.dtype)
+    z1, s1 = L.forward(x)
+    z2, s2 = L.forward(x, save_xg=True)
+    dx1, r1, p1 = L.backward(x, s1, dz)
+    dx2, r2, p2 = L.backward(None, s2, dz)
+    torch.cuda.synchronize()
+    assert np.array_equal(bits(z1), bits(z2))
+    assert np.array_equal(bits(s2.xg), bits(x)[:, inp.permR])
+    for a, b in ((dx1, dx2), (r1, r2), (p1, p2)):
+        assert np.array_equal(bits(a), bits(b))
+
+
 def test_backward_is_deterministic_and_accumulates():
     inp = _inputs("up8b", 512, 1024, 256, 700)
     L = make_layer(inp)
@@ -232,7 +250,7 @@ def test_check_perm_and_errors():
     L = make_layer(inp)
     with pytest.raises(px.PoetxError) as e:
         px.poetx_forward(L.abi(), 16, dev(inp.x, "bf16"), torch.empty((16, 512), dtype=torch.bfloat16,
-                                                                       device="cuda"), None, ws, 64)
+                                                                       device="cuda"), None, None, ws, 64)
     assert e.value.status == 5
 
 
