@@ -132,6 +132,14 @@ poetx_status poetx_layer_cnp_build(const poetx_layer* layer, void* ws, size_t ws
  * order them on one stream or synchronise between them. */
 poetx_status poetx_cnp_build_fixed(int32_t nblk, int32_t b, const float* q, int32_t dtype, void* G, void* stream);
 
+/* The Cayley-Neumann builds of several layers (1 <= nlayers <= 16, all with
+ * the same b and dtype; `layers` is a HOST array of layer structs) in one
+ * batch: GR and GP of every layer.  Workspace:
+ * poetx_layers_cnp_workspace_bytes(nlayers, layers) (0 for an invalid set). */
+size_t poetx_layers_cnp_workspace_bytes(int32_t nlayers, const poetx_layer* layers);
+poetx_status poetx_layers_cnp_build(int32_t nlayers, const poetx_layer* layers, void* ws, size_t ws_bytes,
+                                    void* stream);
+
 /* Backward of poetx_cnp_build: given dG = dL/dG [nblk][b][b] (fp32), writes
  * dq = dL/dq [nblk][b(b-1)/2] (fp32), dq_k = dL/dQ[i][j] - dL/dQ[j][i].
  * accumulate != 0 adds to dq instead of overwriting it.  dtype names the

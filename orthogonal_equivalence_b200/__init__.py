@@ -56,6 +56,8 @@ SIGNATURES = {
     "poetx_cnp_backward": (ctypes.c_int, [_I32, _I32, _VP, _VP, _VP, _I32, _I32, _VP, _SZ, _VP]),
     "poetx_cnp_build_fixed": (ctypes.c_int, [_I32, _I32, _VP, _I32, _VP, _VP]),
     "poetx_layer_cnp_workspace_bytes": (_SZ, [_LP]),
+    "poetx_layers_cnp_workspace_bytes": (_SZ, [_I32, _LP]),
+    "poetx_layers_cnp_build": (ctypes.c_int, [_I32, _LP, _VP, _SZ, _VP]),
     "poetx_layer_cnp_build": (ctypes.c_int, [_LP, _VP, _SZ, _VP]),
     "poetx_forward": (ctypes.c_int, [_LP, _I64, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "poetx_backward": (ctypes.c_int, [_LP, _I64, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I32, _VP, _SZ, _VP]),
@@ -180,6 +182,20 @@ def poetx_layer_cnp_build(layer: poetx_layer, ws, ws_bytes: int, stream=None) ->
            "poetx_layer_cnp_build")
 
 
+def _layer_array(layers):
+    arr = (poetx_layer * len(layers))(*layers)
+    return arr
+
+
+def poetx_layers_cnp_workspace_bytes(layers) -> int:
+    return lib().poetx_layers_cnp_workspace_bytes(len(layers), _layer_array(layers))
+
+
+def poetx_layers_cnp_build(layers, ws, ws_bytes: int, stream=None) -> None:
+    _check(lib().poetx_layers_cnp_build(len(layers), _layer_array(layers), _ptr(ws), ws_bytes, _stream(stream)),
+           "poetx_layers_cnp_build")
+
+
 def poetx_forward(layer: poetx_layer, T: int, x, z, y_save, xg_save, ws, ws_bytes: int, stream=None) -> None:
     _check(lib().poetx_forward(ctypes.byref(layer), T, _ptr(x), _ptr(z), _ptr(y_save), _ptr(xg_save), _ptr(ws),
                                ws_bytes, _stream(stream)), "poetx_forward")
@@ -225,4 +241,4 @@ def poetx_profile_records() -> list:
     return [(names[st[i]], ms[i]) for i in range(n)]
 
 
-from .layer import PoetxLinear  # noqa: E402,F401
+from .layer import LayerGroup, PoetxLinear, Saved  # noqa: E402,F401

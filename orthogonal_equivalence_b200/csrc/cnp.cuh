@@ -62,20 +62,37 @@ __global__ void transpose_blocks_kernel(const T* __restrict__ in, float* __restr
 // Matrices live in row-strided block arrays: block t starts at t * bs, rows
 // ld apart (so a block can sit inside a wider concatenated row).
 
+// Block ranges of up to kMaxSegs sources batched into one launch (the R and
+// P sides of one layer, or of several layers): blocks [start[s], start[s+1])
+// take their packed triangles from q[s] and (for the build) write G to G[s].
+constexpr int kMaxSegs = 32;
+struct Segs {
+  int n;
+  int start[kMaxSegs + 1];
+  const float* q[kMaxSegs];
+  void* G[kMaxSegs];
+};
+
+__device__ __forceinline__ int seg_of(const Segs& sg, int blk) {
+  int s = 0;
+  while (s + 1 < sg.n && blk >= sg.start[s + 1]) ++s;
+  return s;
+}
+
 // Unpack packed triangles into Q (and optionally a second copy).  One block
 // per 32 x 32 tile (ti, tj) with ti <= tj of one b x b block: row i of the
 // tile reads its run of q (contiguous for i < j), writes Q[i][j] = q and,
 // through a shared-memory transpose, the mirrored tile Q[j][i] = -q, so both
 // the reads and the writes are coalesced.  grid (b/32, b/32, nblk), block
 // (32, 8); tiles below the diagonal exit at once.
-__global__ void unpack_skew2_kernel(const float* __restrict__ q0, int n0, const float* __restrict__ q1, int nblk,
-                                    int b, float* __restrict__ o1, int64_t ld1, int64_t bs1, float* __restrict__ o2,
-                                    int64_t ld2, int64_t bs2) {
+__global__ void unpack_skew_kernel(const Segs sg, int nblk, int b, float* __restrict__ o1, int64_t ld1, int64_t bs1,
+                                   float* __restrict__ o2, int64_t ld2, int64_t bs2) {
   __shared__ float tile[32][33];
   const int ti = blockIdx.y, tj = blockIdx.x, blk = blockIdx.z;
   if (ti > tj || blk >= nblk) return;
   const int64_t L = static_cast<int64_t>(b) * (b - 1) / 2;
-  const float* qb = blk < n0 ? q0 + blk * L : q1 + (blk - n0) * L;
+  const int sgi = seg_of(sg, blk);
+  const float* qb = sg.q[sgi] + (blk - sg.start[sgi]) * L;
   float* A1 = o1 + blk * bs1;
   float* A2 = o2 ? o2 + blk * bs2 : nullptr;
   const int r0 = ti * 32, c0 = tj * 32;
@@ -100,6 +117,20 @@ __global__ void unpack_skew2_kernel(const float* __restrict__ q0, int n0, const 
       if (A2) A2[j * ld2 + i] = v;
     }
   }
+}
+
+// Copy contiguous G blocks [nblk][b][b] (elem_bytes each element) to each
+// segment's own G array, 16 bytes per thread.  grid (chunks, nblk).
+__global__ void split_blocks_kernel(const Segs sg, const uint8_t* __restrict__ all, int nblk, int64_t block_bytes) {
+  const int blk = blockIdx.y;
+  if (blk >= nblk) return;
+  const int sgi = seg_of(sg, blk);
+  const uint4* src = reinterpret_cast<const uint4*>(all + blk * block_bytes);
+  uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(sg.G[sgi]) + (blk - sg.start[sgi]) * block_bytes);
+  const int64_t n16 = block_bytes / 16;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n16;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    dst[i] = src[i];
 }
 
 // dG = sum over token splits of the partial products, in split order, for

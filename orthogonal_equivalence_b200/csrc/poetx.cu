@@ -489,19 +489,33 @@ ExtraOut extra_out(float* p, int b, int64_t ld, float cv, bool transposed) {
 
 size_t cnp_units(int32_t nblk, int32_t b) { return al(sizeof(float) * size_t(nblk) * b * b); }
 
-// G0 (n0 blocks) from q0 and G1 (n1 blocks) from q1.
-poetx_status cnp_build2(int32_t b, int32_t dtype, const float* q0, int n0, void* G0, const float* q1, int n1,
-                        void* G1, Carver& ws, cudaStream_t st, int device) {
-  const int nblk = n0 + n1;
+Segs two_segs(const float* q0, int n0, void* G0, const float* q1, int n1, void* G1) {
+  Segs sg{};
+  sg.n = n1 > 0 ? 2 : 1;
+  sg.start[0] = 0;
+  sg.start[1] = n0;
+  sg.start[2] = n0 + n1;
+  sg.q[0] = q0;
+  sg.q[1] = q1;
+  sg.G[0] = G0;
+  sg.G[1] = G1;
+  return sg;
+}
+
+// G of every segment from its packed triangles, all blocks in one batch.
+// Up to two segments write G straight from the GEMM epilogue; more go
+// through a contiguous scratch copy (`gall`, nblk*b*b elements of dtype).
+poetx_status cnp_build_segs(int32_t b, int32_t dtype, const Segs& sg, Carver& ws, cudaStream_t st, int device) {
+  const int nblk = sg.start[sg.n];
   const size_t nbb = size_t(nblk) * b * b;
   float* Q = ws.take<float>(sizeof(float) * nbb);
   float* S = ws.take<float>(sizeof(float) * nbb);
   float* H = ws.take<float>(sizeof(float) * nbb);
+  void* gall = sg.n > 2 ? ws.take<uint8_t>(dtype_size(dtype) * nbb) : nullptr;
   const bool tc_path = use_tc(dtype);
   const int64_t bb = int64_t(b) * b;
   const dim3 ugrid((b + 31) / 32, (b + 31) / 32, nblk), ublock(32, 8);
-  PROFILED(ST_CNP_ELEM, st,
-           unpack_skew2_kernel<<<ugrid, ublock, 0, st>>>(q0, n0, q1, nblk, b, Q, b, bb, nullptr, 0, 0));
+  PROFILED(ST_CNP_ELEM, st, unpack_skew_kernel<<<ugrid, ublock, 0, st>>>(sg, nblk, b, Q, b, bb, nullptr, 0, 0));
   POETX_CUDA(cudaGetLastError());
   // S = -(Q Q^T); H = S + 2Q as a second output
   {
@@ -517,15 +531,31 @@ poetx_status cnp_build2(int32_t b, int32_t dtype, const float* q0, int n0, void*
   // G = H S^T + 2Q + 2S + I  (S^T = S)
   {
     GemmDesc g = cat_nt_desc(H, S, nblk, b, b, b, 1.f);
-    g.C = out_blocks(G0, elem_type(dtype), b, b);
-    g.C.ptr2 = G1;
-    g.C.split_batch = n0;
+    if (gall) {
+      g.C = out_blocks(gall, elem_type(dtype), b, b);
+    } else {
+      g.C = out_blocks(sg.G[0], elem_type(dtype), b, b);
+      g.C.ptr2 = sg.G[1];
+      g.C.split_batch = sg.start[1];
+    }
     g.add1 = add_view(Q, b, b, 2.f);
     g.add2 = add_view(S, b, b, 2.f);
     g.diag = 1.f;
     PROFILED(ST_CNP_GEMM, st, POETX_CUDA(launch_gemm(g, tc_path, st, device)));
   }
+  if (gall) {
+    const int64_t block_bytes = int64_t(dtype_size(dtype)) * bb;
+    const dim3 grid(static_cast<unsigned>((block_bytes / 16 + 255) / 256), nblk);
+    PROFILED(ST_CNP_ELEM, st,
+             split_blocks_kernel<<<grid, 256, 0, st>>>(sg, static_cast<const uint8_t*>(gall), nblk, block_bytes));
+    POETX_CUDA(cudaGetLastError());
+  }
   return POETX_OK;
+}
+
+poetx_status cnp_build2(int32_t b, int32_t dtype, const float* q0, int n0, void* G0, const float* q1, int n1,
+                        void* G1, Carver& ws, cudaStream_t st, int device) {
+  return cnp_build_segs(b, dtype, two_segs(q0, n0, G0, q1, n1, G1), ws, st, device);
 }
 
 // dq from dG for G = I + 2A + 2S + H S with S = A A, H = 2A + S:
@@ -554,7 +584,8 @@ poetx_status cnp_backward2(int32_t b, int32_t dtype, const float* q0, int n0, co
   // A -> X2[:, b:2b] and Y2[:, 0:b]
   const dim3 ugrid((b + 31) / 32, (b + 31) / 32, nblk), ublock(32, 8);
   PROFILED(ST_CNP_ELEM, st,
-           unpack_skew2_kernel<<<ugrid, ublock, 0, st>>>(q0, n0, q1, nblk, b, X2 + b, b3, b * b3, Y2, b3, b * b3));
+           unpack_skew_kernel<<<ugrid, ublock, 0, st>>>(two_segs(q0, n0, nullptr, q1, n1, nullptr), nblk, b, X2 + b,
+                                                        b3, b * b3, Y2, b3, b * b3));
   // dG -> X1[:, b:2b], X2[:, 2b:3b];  dG^T -> Y1[:, 0:b]
   {
     const dim3 grid((b + 31) / 32, (b + 31) / 32, nblk), block(32, 8);
@@ -635,6 +666,49 @@ size_t poetx_cnp_workspace_bytes(int32_t nblk, int32_t b, int32_t dtype) {
   (void)dtype;
   if (nblk <= 0 || b < 2) return 0;
   return kAlign + cnp_bwd_ws(nblk, b);
+}
+
+size_t poetx_layers_cnp_workspace_bytes(int32_t nlayers, const poetx_layer* layers) {
+  if (nlayers < 1 || 2 * nlayers > kMaxSegs || !layers) return 0;
+  int64_t nblk = 0;
+  for (int i = 0; i < nlayers; ++i) {
+    if (check_layer(&layers[i]) != POETX_OK || layers[i].b != layers[0].b || layers[i].dtype != layers[0].dtype)
+      return 0;
+    nblk += layers[i].m / layers[i].b + layers[i].n / layers[i].b;
+  }
+  const int b = layers[0].b;
+  return kAlign + 3 * cnp_units(static_cast<int32_t>(nblk), b) +
+         al(size_t(dtype_size(layers[0].dtype)) * size_t(nblk) * b * b);
+}
+
+poetx_status poetx_layers_cnp_build(int32_t nlayers, const poetx_layer* layers, void* ws, size_t ws_bytes,
+                                    void* stream) {
+  if (nlayers < 1 || 2 * nlayers > kMaxSegs || !layers) return POETX_E_ARG;
+  for (int i = 0; i < nlayers; ++i) {
+    POETX_TRY(check_layer(&layers[i]));
+    if (layers[i].b != layers[0].b) return POETX_E_SHAPE;
+    if (layers[i].dtype != layers[0].dtype) return POETX_E_DTYPE;
+  }
+  if (!ws || ws_bytes < poetx_layers_cnp_workspace_bytes(nlayers, layers)) return POETX_E_WORKSPACE;
+  int dev;
+  POETX_TRY(current_device(&dev));
+  Segs sg{};
+  sg.n = 2 * nlayers;
+  int blk = 0;
+  for (int i = 0; i < nlayers; ++i) {
+    const poetx_layer& L = layers[i];
+    sg.start[2 * i] = blk;
+    sg.q[2 * i] = L.qR;
+    sg.G[2 * i] = L.GR;
+    blk += L.m / L.b;
+    sg.start[2 * i + 1] = blk;
+    sg.q[2 * i + 1] = L.qP;
+    sg.G[2 * i + 1] = L.GP;
+    blk += L.n / L.b;
+  }
+  sg.start[sg.n] = blk;
+  Carver c(ws, ws_bytes);
+  return cnp_build_segs(layers[0].b, layers[0].dtype, sg, c, static_cast<cudaStream_t>(stream), dev);
 }
 
 size_t poetx_layer_cnp_workspace_bytes(const poetx_layer* layer) {

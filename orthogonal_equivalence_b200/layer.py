@@ -14,7 +14,8 @@ import torch
 
 from . import (POETX_BF16, POETX_FP32, make_layer, poetx_backward, poetx_backward_workspace_bytes,
                poetx_forward, poetx_forward_workspace_bytes, poetx_frame_export, poetx_frame_import,
-               poetx_layer_cnp_build, poetx_layer_cnp_workspace_bytes, poetx_merge, poetx_merge_workspace_bytes)
+               poetx_layer_cnp_build, poetx_layer_cnp_workspace_bytes, poetx_layers_cnp_build,
+               poetx_layers_cnp_workspace_bytes, poetx_merge, poetx_merge_workspace_bytes)
 
 _TORCH_DTYPE = {POETX_BF16: torch.bfloat16, POETX_FP32: torch.float32}
 
@@ -139,3 +140,19 @@ class PoetxLinear:
         self.W = W_out
         self.permR.copy_(newR)
         self.permP.copy_(newP)
+
+
+class LayerGroup:
+    """Several layers with the same b and dtype whose G blocks are rebuilt
+    together (one batched CNP build for all of them)."""
+
+    def __init__(self, layers):
+        self.layers = list(layers)
+        self._ws = None
+
+    def build(self, stream=None) -> None:
+        abis = [L.abi() for L in self.layers]
+        nb = poetx_layers_cnp_workspace_bytes(abis)
+        if self._ws is None or self._ws.numel() < nb:
+            self._ws = torch.empty(max(nb, 1), dtype=torch.uint8, device=self.layers[0].device)
+        poetx_layers_cnp_build(abis, self._ws, nb, stream)

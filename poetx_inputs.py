@@ -139,9 +139,10 @@ def layer_inputs(cfg: Config, layer: int = 0, T: int | None = None, m: int | Non
                  zero_q: bool = False) -> LayerInputs:
     """Draw one layer's inputs.  Overrides (T, m, n, b) give reduced shapes of
     the same recipe for parity tests; the full configuration is the default."""
-    _, m0, n0 = cfg.layers[layer]
-    m = m0 if m is None else m
-    n = n0 if n is None else n
+    if m is None or n is None:
+        _, m0, n0 = cfg.layers[layer]
+        m = m0 if m is None else m
+        n = n0 if n is None else n
     b = cfg.b if b is None else b
     T = cfg.T if T is None else T
     sq = cfg.sigma_q if sigma_q is None else sigma_q

@@ -106,6 +106,26 @@ def test_cnp_build_and_backward_parity(dtype, b, nblk):
     check(host64(dq), 2 * dqo, dtype, "dq accumulated")
 
 
+@pytest.mark.parametrize("name", ["block8b", "tiny"])
+def test_batched_build_of_several_layers(name):
+    # one CNP build for the R and P blocks of several layers equals the
+    # per-layer builds and the oracle
+    cfg = pi.CONFIGS[name]
+    shapes = [(512, 256), (256, 768), (1024, 512)] if name == "block8b" else [(128, 192), (256, 64)]
+    inps = [_inputs(name, m, n, None, 8, layer=k) for k, (m, n) in enumerate(shapes)]
+    Ls = [make_layer(i) for i in inps]
+    ref = [(L.GR.clone(), L.GP.clone()) for L in Ls]
+    for L in Ls:
+        L.GR.zero_()
+        L.GP.zero_()
+    px.LayerGroup(Ls).build()
+    torch.cuda.synchronize()
+    for L, inp, (gr, gp) in zip(Ls, inps, ref):
+        assert np.array_equal(bits(L.GR), bits(gr)) and np.array_equal(bits(L.GP), bits(gp))
+        check(host64(L.GR), oracle.cnp_blocks(inp.qR, inp.b), inp.dtype, "GR")
+        check(host64(L.GP), oracle.cnp_blocks(inp.qP, inp.b), inp.dtype, "GP")
+
+
 @pytest.mark.parametrize("dtype", ["fp32", "bf16"])
 def test_zero_q_gives_identity_and_plain_linear(dtype):
     name = "tiny" if dtype == "fp32" else "attn3b"
