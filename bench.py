@@ -336,6 +336,53 @@ def bench_poetx(args, cfg: pi.Config) -> dict:
         e2e = {"value": world * cfg.T * e_steps / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "steps": e_steps,
                "h2d_gbs": h2d * e_steps / (e_ms / 1e3) / 1e9}
+    # Variants of the same step (see the POET-X write-up's three variants and
+    # its optimizer): "mem" keeps nothing between forward and backward but x
+    # (the backward recomputes Y); "xq" keeps the frozen weights as int8 codes
+    # and dequantizes each one into a shared scratch before every use; the
+    # optimizer step is AdamW on all packed triangles plus the batched CNP
+    # rebuild.
+    variants = None
+    if not args.no_variants:
+        def timed(fn, k):
+            barrier(device)
+            a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(k):
+                fn()
+            b_.record(stream)
+            torch.cuda.synchronize(device)
+            barrier(device)
+            return reduce_max(a.elapsed_time(b_), device) / k
+
+        def step_mem():
+            layers[0]["group"].build()
+            for l in layers:
+                l["L"].forward(l["x"], save=False, z=l["z"])
+            for l in reversed(layers):
+                l["L"].backward(l["x"], None, l["dz"], dx=l["dx"], dqR=l["dqR"], dqP=l["dqP"])
+            allreduce_grads(flat)
+
+        variants = {}
+        step_mem()
+        ms = timed(step_mem, args.steps)
+        variants["mem"] = {"tokens_per_s": world * cfg.T / (ms / 1e3), "ms_per_step": ms,
+                           "note": "backward recomputes Y; no [T][n] activation kept"}
+        group = layers[0]["group"]
+        group.flatten_params()
+        opt = lambda: group.optimizer_step(flat, 1e-4, weight_decay=0.0)  # noqa: E731
+        opt()
+        ms = timed(opt, args.steps)
+        variants["optimizer_step"] = {"ms_per_step": ms, "params": int(group.q.numel()),
+                                      "note": "AdamW on every packed triangle + batched CNP rebuild of every G"}
+        scratch = torch.empty(max(l["m"] * l["n"] for l in layers), dtype=torch.bfloat16, device=device)
+        for l in layers:
+            l["L"].quantize_weight(scratch)
+        run_step(layers, flat)
+        ms = timed(lambda: run_step(layers, flat), args.steps)
+        variants["xq"] = {"tokens_per_s": world * cfg.T / (ms / 1e3), "ms_per_step": ms,
+                          "weight_bytes": int(sum(l["m"] * l["n"] + 4 * l["n"] for l in layers)),
+                          "note": "int8 per-row weights, dequantized into one shared scratch before each use"}
     device_error = px.poetx_device_error()
 
     peaks, peak_src = measured_peaks()
@@ -392,6 +439,7 @@ def bench_poetx(args, cfg: pi.Config) -> dict:
         "gpu_launches": total_launches,
         "clocks": clocks,
         "e2e": e2e,
+        "variants": variants,
         "device_error": device_error,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -475,6 +523,7 @@ def main(argv=None):
                     help="override the workload's tokens per GPU (smaller cases for profiler captures)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-variants", action="store_true", help="skip the mem / xq / optimizer-step timings")
     ap.add_argument("--cpu-tokens", type=int, default=512, help="token sample of the CPU-baseline leg")
     ap.add_argument("--ref-tokens", type=int, default=64, help="token sample per step of --impl reference")
     args = ap.parse_args(argv)

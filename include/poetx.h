@@ -92,6 +92,7 @@ poetx_status poetx_device_error(uint32_t* code);
 size_t poetx_cnp_workspace_bytes(int32_t nblk, int32_t b, int32_t dtype);
 size_t poetx_forward_workspace_bytes(const poetx_layer* layer, int64_t T);
 size_t poetx_backward_workspace_bytes(const poetx_layer* layer, int64_t T);
+size_t poetx_backward_recompute_workspace_bytes(const poetx_layer* layer, int64_t T);
 size_t poetx_merge_workspace_bytes(const poetx_layer* layer);
 size_t poetx_check_perm_workspace_bytes(int32_t len);
 
@@ -159,10 +160,14 @@ poetx_status poetx_forward(const poetx_layer* layer, int64_t T, const void* x, v
 
 /* Backward of L = <dz, z>: dx [T][m] (dtype; NULL skips it) and the packed
  * gradients dqR [m/b][b(b-1)/2], dqP [n/b][b(b-1)/2] (fp32; overwritten, or
- * added to when accumulate != 0).  Needs the y_save of the matching forward
- * and either its xg_save or (xg_save == NULL) the input x, which is then
- * gathered again; W0 is frozen, so no dW0.  The dq sums over tokens use a
- * fixed split and order (deterministic for a given shape). */
+ * added to when accumulate != 0).  Needs either the xg_save of the matching
+ * forward or (xg_save == NULL) the input x, which is then gathered again, and
+ * the forward's y_save.  With y_save == NULL the backward recomputes Y from
+ * Xg (one more block product and W0 product; the "POET-X mem" variant of the
+ * write-up's section "三种变体", which keeps no [T][n] activation); its
+ * workspace is then poetx_backward_recompute_workspace_bytes.  W0 is frozen,
+ * so no dW0.  The dq sums over tokens use a fixed split and order
+ * (deterministic for a given shape). */
 poetx_status poetx_backward(const poetx_layer* layer, int64_t T, const void* x, const void* y_save,
                             const void* xg_save, const void* dz, void* dx, float* dqR, float* dqP,
                             int32_t accumulate, void* ws, size_t ws_bytes, void* stream);
@@ -182,11 +187,33 @@ poetx_status poetx_merge(const poetx_layer* layer, const int32_t* new_permR, con
 poetx_status poetx_check_perm(const int32_t* perm, int32_t len, int32_t* d_ok, void* ws, size_t ws_bytes,
                               void* stream);
 
+/* POET-XQ storage of the frozen weight (write-up section "POET-XQ"): the
+ * base weight is kept quantized and dequantized at run time.  The pages fix no
+ * format; the reading here is int8, symmetric, one fp32 scale per row of the
+ * stored [n][m] weight (per output feature): scale = max|row| / 127, code =
+ * round-half-even(w / scale) clamped to [-127, 127] (fp32 arithmetic).
+ * quantize: W [n][m] (dtype) -> Wq [n][m] int8 + scale [n] fp32.
+ * dequantize: w = code * scale (fp32 product) rounded once to dtype, into W;
+ * run it into a scratch weight before poetx_forward / poetx_backward. */
+poetx_status poetx_weight_quantize(int32_t n, int32_t m, const void* W, int32_t dtype, int8_t* Wq, float* scale,
+                                   void* stream);
+poetx_status poetx_weight_dequantize(int32_t n, int32_t m, const int8_t* Wq, const float* scale, int32_t dtype,
+                                     void* W, void* stream);
+
+/* Optimizer step on packed triangles (fp32, n entries): AdamW with decoupled
+ * weight decay (the write-up names get_poet_optimizer without describing it;
+ * AdamW is the reading taken): m1 <- b1 m1 + (1-b1) g; m2 <- b2 m2 + (1-b2) g^2;
+ * q <- q (1 - lr wd) - lr (m1 / (1 - b1^step)) / (sqrt(m2 / (1 - b2^step)) + eps).
+ * step >= 1 counts the updates so far including this one.  After it, rebuild
+ * G (poetx_layers_cnp_build). */
+poetx_status poetx_adamw_step(int64_t n, float* q, const float* grad, float* m1, float* m2, float lr, float beta1,
+                              float beta2, float eps, float weight_decay, int32_t step, void* stream);
+
 /* Stage profiler (tracing).  Between poetx_profile_begin() and
  * poetx_profile_end(), every kernel the library queues is bracketed by a pair
  * of CUDA events on its stream and tagged with its stage (permute,
  * blockdiag_gemm, w0_gemm, dg_gemm, cnp_gemm, cnp_elementwise, dg_reduce,
- * merge).  poetx_profile_end waits for the recorded events, writes the summed
+ * merge, dequant, optimizer).  poetx_profile_end waits for the recorded events, writes the summed
  * device time in ms (HOST array ms_per_stage[nstages]) and the number of
  * launches (HOST array launches_per_stage[nstages]) per stage, and stops
  * recording.  The events are created on first use and reused. */

@@ -37,7 +37,8 @@ is T x n.  All arithmetic is float64; numpy's matmul is the only library
 primitive used.
 
 Parity: every function here is pinned by tests against closed forms,
-invariants, brute force or finite differences; none is "parity unpinned".
+invariants, brute force, finite differences or a library routine (the AdamW
+step against torch.optim.AdamW); none is "parity unpinned".
 """
 from __future__ import annotations
 
@@ -308,3 +309,55 @@ def from_frame(Wf: np.ndarray, permR, permP) -> np.ndarray:
     out = np.empty_like(Wf)
     out[np.ix_(np.asarray(permP, dtype=np.int64), np.asarray(permR, dtype=np.int64))] = Wf
     return out
+
+
+# --------------------------------------------------------------------------
+# POET-XQ (section "POET-XQ"): the base weight stored quantized, dequantized
+# at run time.  Reading: int8, symmetric, one scale per row of the stored
+# [n][m] weight; the scale and the codes are decided in float32 arithmetic
+# (scale = max|row| / 127, code = round-half-even(w / scale) clamped to
+# [-127, 127]); w = code * scale in float32, rounded once to the weight dtype.
+# --------------------------------------------------------------------------
+
+
+def quantize_rows(W: np.ndarray):
+    """[n][m] weight values -> (int8 codes [n][m], float32 scales [n])."""
+    W32 = np.asarray(W, dtype=np.float32)
+    amax = np.max(np.abs(W32), axis=1)
+    scale = (amax / np.float32(127.0)).astype(np.float32)
+    codes = np.zeros(W32.shape, dtype=np.int8)
+    nz = scale > 0
+    q = np.rint(W32[nz] / scale[nz, None]).astype(np.float32)
+    codes[nz] = np.clip(q, -127, 127).astype(np.int8)
+    return codes, scale
+
+
+def dequantize_rows(codes: np.ndarray, scale: np.ndarray) -> np.ndarray:
+    """code * scale as the float32 product (float32 array)."""
+    return codes.astype(np.float32) * np.asarray(scale, dtype=np.float32)[:, None]
+
+
+def round_to_bf16(a: np.ndarray) -> np.ndarray:
+    """float32 values rounded to bfloat16 (round to nearest even), returned as
+    float64 values."""
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32)
+    r = ((u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)) << np.uint32(16)
+    return r.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+# --------------------------------------------------------------------------
+# Optimizer step on the packed triangles (get_poet_optimizer in the API
+# snippet is not described; reading: AdamW with decoupled weight decay).
+# --------------------------------------------------------------------------
+
+
+def adamw_step(q, g, m, v, lr, beta1, beta2, eps, weight_decay, step):
+    """One AdamW update in float64; returns (q, m, v)."""
+    q = np.asarray(q, dtype=np.float64)
+    g = np.asarray(g, dtype=np.float64)
+    m = beta1 * np.asarray(m, dtype=np.float64) + (1.0 - beta1) * g
+    v = beta2 * np.asarray(v, dtype=np.float64) + (1.0 - beta2) * g * g
+    m_hat = m / (1.0 - beta1 ** step)
+    v_hat = v / (1.0 - beta2 ** step)
+    q = q * (1.0 - lr * weight_decay) - lr * m_hat / (np.sqrt(v_hat) + eps)
+    return q, m, v

@@ -48,6 +48,7 @@ SIGNATURES = {
     "poetx_cnp_workspace_bytes": (_SZ, [_I32, _I32, _I32]),
     "poetx_forward_workspace_bytes": (_SZ, [_LP, _I64]),
     "poetx_backward_workspace_bytes": (_SZ, [_LP, _I64]),
+    "poetx_backward_recompute_workspace_bytes": (_SZ, [_LP, _I64]),
     "poetx_merge_workspace_bytes": (_SZ, [_LP]),
     "poetx_check_perm_workspace_bytes": (_SZ, [_I32]),
     "poetx_frame_import": (ctypes.c_int, [_LP, _VP, _VP]),
@@ -63,6 +64,10 @@ SIGNATURES = {
     "poetx_backward": (ctypes.c_int, [_LP, _I64, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I32, _VP, _SZ, _VP]),
     "poetx_merge": (ctypes.c_int, [_LP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "poetx_check_perm": (ctypes.c_int, [_VP, _I32, _VP, _VP, _SZ, _VP]),
+    "poetx_weight_quantize": (ctypes.c_int, [_I32, _I32, _VP, _I32, _VP, _VP, _VP]),
+    "poetx_weight_dequantize": (ctypes.c_int, [_I32, _I32, _VP, _VP, _I32, _VP, _VP]),
+    "poetx_adamw_step": (ctypes.c_int, [_I64, _VP, _VP, _VP, _VP, ctypes.c_float, ctypes.c_float, ctypes.c_float,
+                                        ctypes.c_float, ctypes.c_float, _I32, _VP]),
     "poetx_profile_stage_count": (_I32, []),
     "poetx_profile_stage_name": (ctypes.c_char_p, [_I32]),
     "poetx_profile_begin": (ctypes.c_int, []),
@@ -141,6 +146,10 @@ def poetx_backward_workspace_bytes(layer: poetx_layer, T: int) -> int:
     return lib().poetx_backward_workspace_bytes(ctypes.byref(layer), T)
 
 
+def poetx_backward_recompute_workspace_bytes(layer: poetx_layer, T: int) -> int:
+    return lib().poetx_backward_recompute_workspace_bytes(ctypes.byref(layer), T)
+
+
 def poetx_merge_workspace_bytes(layer: poetx_layer) -> int:
     return lib().poetx_merge_workspace_bytes(ctypes.byref(layer))
 
@@ -216,6 +225,22 @@ def poetx_merge(layer: poetx_layer, new_permR, new_permP, W_out, ws, ws_bytes: i
 def poetx_check_perm(perm, length: int, d_ok, ws, ws_bytes: int, stream=None) -> None:
     _check(lib().poetx_check_perm(_ptr(perm), length, _ptr(d_ok), _ptr(ws), ws_bytes, _stream(stream)),
            "poetx_check_perm")
+
+
+def poetx_weight_quantize(n: int, m: int, W, dtype: int, Wq, scale, stream=None) -> None:
+    _check(lib().poetx_weight_quantize(n, m, _ptr(W), dtype, _ptr(Wq), _ptr(scale), _stream(stream)),
+           "poetx_weight_quantize")
+
+
+def poetx_weight_dequantize(n: int, m: int, Wq, scale, dtype: int, W, stream=None) -> None:
+    _check(lib().poetx_weight_dequantize(n, m, _ptr(Wq), _ptr(scale), dtype, _ptr(W), _stream(stream)),
+           "poetx_weight_dequantize")
+
+
+def poetx_adamw_step(n: int, q, grad, m1, m2, lr: float, beta1: float, beta2: float, eps: float,
+                     weight_decay: float, step: int, stream=None) -> None:
+    _check(lib().poetx_adamw_step(n, _ptr(q), _ptr(grad), _ptr(m1), _ptr(m2), lr, beta1, beta2, eps, weight_decay,
+                                  step, _stream(stream)), "poetx_adamw_step")
 
 
 def poetx_profile_begin() -> None:

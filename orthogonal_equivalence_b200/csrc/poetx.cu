@@ -7,6 +7,7 @@
 // centric layer), 2 (block-stochastic R, P), 3 (Cayley-Neumann blocks,
 // packed triangle) and the merge_if_needed step of its API snippet.
 #include <cstdint>
+#include <cmath>
 #include <cstring>
 #include <mutex>
 #include <utility>
@@ -16,6 +17,8 @@
 #include "cnp.cuh"
 #include "gemm_host.cuh"
 #include "perm.cuh"
+#include "quant.cuh"
+#include "adamw.cuh"
 
 using namespace poetx;
 
@@ -115,10 +118,12 @@ enum Stage : int {
   ST_CNP_ELEM,
   ST_REDUCE,
   ST_MERGE,
+  ST_DEQUANT,
+  ST_OPTIM,
   ST_COUNT
 };
-const char* const kStageNames[ST_COUNT] = {"permute",  "blockdiag_gemm",  "w0_gemm",   "dg_gemm",
-                                           "cnp_gemm", "cnp_elementwise", "dg_reduce", "merge"};
+const char* const kStageNames[ST_COUNT] = {"permute",  "blockdiag_gemm",  "w0_gemm",   "dg_gemm", "cnp_gemm",
+                                           "cnp_elementwise", "dg_reduce", "merge", "dequant", "optimizer"};
 
 struct Profiler {
   std::mutex mu;
@@ -210,6 +215,12 @@ size_t bwd_ws(const poetx_layer* L, int64_t T) {
   return kAlign + 2 * al(es * T * mx) + al(es * T * L->m) +
          al(sizeof(float) * dg_splits(nP, L->b, T, L->dtype) * nP * bb) +
          al(sizeof(float) * dg_splits(nR, L->b, T, L->dtype) * nR * bb) + cnp_bwd_ws(nR + nP, L->b);
+}
+
+// The backward that recomputes Y (y_save == NULL) also needs Y [T][n] and Xg [T][m].
+size_t bwd_recompute_ws(const poetx_layer* L, int64_t T) {
+  const size_t es = dtype_size(L->dtype);
+  return bwd_ws(L, T) + al(es * T * L->n) + al(es * T * L->m);
 }
 
 size_t merge_ws(const poetx_layer* L) {
@@ -737,6 +748,11 @@ size_t poetx_backward_workspace_bytes(const poetx_layer* layer, int64_t T) {
   return bwd_ws(layer, T);
 }
 
+size_t poetx_backward_recompute_workspace_bytes(const poetx_layer* layer, int64_t T) {
+  if (check_layer(layer) != POETX_OK || T < 0) return 0;
+  return bwd_recompute_ws(layer, T);
+}
+
 size_t poetx_merge_workspace_bytes(const poetx_layer* layer) {
   if (check_layer(layer) != POETX_OK) return 0;
   return merge_ws(layer);
@@ -877,11 +893,12 @@ poetx_status poetx_backward(const poetx_layer* layer, int64_t T, const void* x, 
     return POETX_OK;
   }
   if (!xg_save) POETX_TRY(check_ptr(x));
-  POETX_TRY(check_ptr(y_save));
+  if (y_save && !aligned16(y_save)) return POETX_E_ALIGN;
   POETX_TRY(check_ptr(dz));
   if (xg_save && !aligned16(xg_save)) return POETX_E_ALIGN;
   if (dx && !aligned16(dx)) return POETX_E_ALIGN;
-  if (!ws || ws_bytes < bwd_ws(layer, T)) return POETX_E_WORKSPACE;
+  const bool recompute = y_save == nullptr;
+  if (!ws || ws_bytes < (recompute ? bwd_recompute_ws(layer, T) : bwd_ws(layer, T))) return POETX_E_WORKSPACE;
   int dev;
   POETX_TRY(current_device(&dev));
   const int et = elem_type(L.dtype);
@@ -896,6 +913,38 @@ poetx_status poetx_backward(const poetx_layer* layer, int64_t T, const void* x, 
   void* dU = c.take<uint8_t>(es * T * L.m);
   float* partP = c.take<float>(sizeof(float) * sP * nP * bb);
   float* partR = c.take<float>(sizeof(float) * sR * nR * bb);
+
+  if (recompute) {
+    // "mem" variant: Y was not kept; recompute it from x (Xg, U = Xg Diag(G_R), Y = U W~)
+    void* Ybuf = c.take<uint8_t>(es * T * L.n);
+    void* Xbuf = c.take<uint8_t>(es * T * L.m);
+    if (!xg_save) {
+      PROFILED(ST_PERMUTE, st, POETX_CUDA(permute_dt(L.dtype, x, Xbuf, T, L.m, L.permR, 0, st, dev)));
+      xg_save = Xbuf;
+    }
+    void* U = dU;  // dU is written only later
+    PROFILED(ST_BLOCKDIAG, st, POETX_CUDA(launch_gemm(blockdiag_desc(xg_save, et, T, L.m, L.b, L.GR, false, U, et), tc_path, st, dev)));
+    GemmDesc g;
+    g.M = static_cast<int>(T);
+    g.N = L.n;
+    g.K = L.m;
+    g.A = colblocks_view(U, et, T, L.m, 0);
+    Operand2D b;
+    b.ptr = L.W;
+    b.et = et;
+    b.rows = L.n;
+    b.cols = L.m;
+    b.ld = L.m;
+    b.mn_major = false;
+    g.B = b;
+    g.C.ptr = Ybuf;
+    g.C.et = et;
+    g.C.ld = L.n;
+    g.C.view_rows = T;
+    g.C.view_cols = L.n;
+    PROFILED(ST_W0, st, POETX_CUDA(launch_gemm(g, tc_path, st, dev)));
+    y_save = Ybuf;
+  }
 
   // dV = dz Psi_P^T
   void* dV = bufA;
@@ -1186,4 +1235,75 @@ extern "C" poetx_status poetx_cnp_build_fixed(int32_t nblk, int32_t b, const flo
   // Q, S and H are written in full before they are read: nothing to clear.
   Carver c(scratch, kFixedScratchBytes);
   return cnp_build2(b, dtype, q, nblk, G, nullptr, 0, nullptr, c, static_cast<cudaStream_t>(stream), dev);
+}
+
+// ---------------------------------------------------------------- POET-XQ weight storage
+extern "C" poetx_status poetx_weight_quantize(int32_t n, int32_t m, const void* W, int32_t dtype, int8_t* Wq,
+                                              float* scale, void* stream) {
+  if (dtype != POETX_FP32 && dtype != POETX_BF16) return POETX_E_DTYPE;
+  if (n < 0 || m <= 0) return POETX_E_ARG;
+  if (n == 0) return POETX_OK;
+  POETX_TRY(check_ptr(W));
+  POETX_TRY(check_ptr(Wq));
+  POETX_TRY(check_ptr(scale));
+  int dev;
+  POETX_TRY(current_device(&dev));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int grid = n < sm_count(dev) * 8 ? n : sm_count(dev) * 8;
+  if (dtype == POETX_BF16)
+    quantize_rows_kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(W), n, m, Wq, scale);
+  else
+    quantize_rows_kernel<<<grid, 256, 0, st>>>(static_cast<const float*>(W), n, m, Wq, scale);
+  POETX_CUDA(cudaGetLastError());
+  return POETX_OK;
+}
+
+extern "C" poetx_status poetx_weight_dequantize(int32_t n, int32_t m, const int8_t* Wq, const float* scale,
+                                                int32_t dtype, void* W, void* stream) {
+  if (dtype != POETX_FP32 && dtype != POETX_BF16) return POETX_E_DTYPE;
+  if (n < 0 || m <= 0) return POETX_E_ARG;
+  if (n == 0) return POETX_OK;
+  POETX_TRY(check_ptr(W));
+  POETX_TRY(check_ptr(Wq));
+  POETX_TRY(check_ptr(scale));
+  int dev;
+  POETX_TRY(current_device(&dev));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t total = int64_t(n) * m;
+  if (dtype == POETX_BF16 && m % 16 == 0) {
+    PROFILED(ST_DEQUANT, st,
+             dequantize_rows_bf16x16_kernel<<<grid_for(total / 16, 256, dev), 256, 0, st>>>(
+                 Wq, scale, n, m, static_cast<__nv_bfloat16*>(W)));
+  } else if (dtype == POETX_BF16) {
+    PROFILED(ST_DEQUANT, st,
+             dequantize_rows_kernel<<<grid_for(total, 256, dev), 256, 0, st>>>(Wq, scale, n, m,
+                                                                              static_cast<__nv_bfloat16*>(W)));
+  } else {
+    PROFILED(ST_DEQUANT, st,
+             dequantize_rows_kernel<<<grid_for(total, 256, dev), 256, 0, st>>>(Wq, scale, n, m, static_cast<float*>(W)));
+  }
+  POETX_CUDA(cudaGetLastError());
+  return POETX_OK;
+}
+
+// ---------------------------------------------------------------- optimizer step on packed q
+extern "C" poetx_status poetx_adamw_step(int64_t n, float* q, const float* grad, float* m1, float* m2, float lr,
+                                         float beta1, float beta2, float eps, float weight_decay, int32_t step,
+                                         void* stream) {
+  if (n < 0 || step < 1) return POETX_E_ARG;
+  if (n == 0) return POETX_OK;
+  POETX_TRY(check_ptr(q));
+  POETX_TRY(check_ptr(grad));
+  POETX_TRY(check_ptr(m1));
+  POETX_TRY(check_ptr(m2));
+  int dev;
+  POETX_TRY(current_device(&dev));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const float bc1 = static_cast<float>(1.0 - std::pow(static_cast<double>(beta1), step));
+  const float bc2 = static_cast<float>(1.0 - std::pow(static_cast<double>(beta2), step));
+  PROFILED(ST_OPTIM, st,
+           adamw_kernel<<<grid_for((n + 3) / 4, 256, dev), 256, 0, st>>>(n, q, grad, m1, m2, lr, beta1, beta2, eps,
+                                                                         weight_decay, bc1, bc2));
+  POETX_CUDA(cudaGetLastError());
+  return POETX_OK;
 }

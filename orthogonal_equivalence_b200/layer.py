@@ -12,10 +12,12 @@ from typing import NamedTuple, Optional, Tuple
 
 import torch
 
-from . import (POETX_BF16, POETX_FP32, make_layer, poetx_backward, poetx_backward_workspace_bytes,
+from . import (POETX_BF16, POETX_FP32, make_layer, poetx_backward, poetx_backward_recompute_workspace_bytes,
+               poetx_backward_workspace_bytes,
                poetx_forward, poetx_forward_workspace_bytes, poetx_frame_export, poetx_frame_import,
                poetx_layer_cnp_build, poetx_layer_cnp_workspace_bytes, poetx_layers_cnp_build,
-               poetx_layers_cnp_workspace_bytes, poetx_merge, poetx_merge_workspace_bytes)
+               poetx_layers_cnp_workspace_bytes, poetx_merge, poetx_merge_workspace_bytes, poetx_weight_dequantize,
+               poetx_weight_quantize, poetx_adamw_step)
 
 _TORCH_DTYPE = {POETX_BF16: torch.bfloat16, POETX_FP32: torch.float32}
 
@@ -23,7 +25,7 @@ _TORCH_DTYPE = {POETX_BF16: torch.bfloat16, POETX_FP32: torch.float32}
 class Saved(NamedTuple):
     """Activations the forward keeps for the backward: Y ([T][n], the P-side
     input in the Psi_P frame) and optionally Xg ([T][m], x in the Psi_R frame)."""
-    y: torch.Tensor
+    y: Optional[torch.Tensor]
     xg: Optional[torch.Tensor]
 
 
@@ -45,6 +47,28 @@ class PoetxLinear:
         self.GR = torch.empty((m // b, b, b), dtype=td, device=self.device)
         self.GP = torch.empty((n // b, b, b), dtype=td, device=self.device)
         self._ws = {}
+        self.Wq = None      # POET-XQ: int8 codes of W and per-row scales
+        self.Wscale = None
+        self._wscratch = None
+
+    # -------------------------------------------------------------- POET-XQ
+    def quantize_weight(self, scratch: Optional[torch.Tensor] = None, stream=None) -> None:
+        """Keep W as int8 codes + per-row scales (POET-XQ) and drop the bf16
+        copy; every forward / backward dequantizes it into `scratch` (a flat
+        tensor of at least n*m elements of the layer dtype, which several
+        layers may share) right before use."""
+        self.Wq = torch.empty((self.n, self.m), dtype=torch.int8, device=self.device)
+        self.Wscale = torch.empty(self.n, dtype=torch.float32, device=self.device)
+        poetx_weight_quantize(self.n, self.m, self.W, self.dtype, self.Wq, self.Wscale, stream)
+        if scratch is None:
+            scratch = torch.empty(self.n * self.m, dtype=self.torch_dtype, device=self.device)
+        self._wscratch = scratch
+        self.W = scratch[: self.n * self.m].view(self.n, self.m)
+
+    def _dequantize(self, stream=None) -> None:
+        if self.Wq is not None:
+            self.W = self._wscratch[: self.n * self.m].view(self.n, self.m)
+            poetx_weight_dequantize(self.n, self.m, self.Wq, self.Wscale, self.dtype, self.W, stream)
 
     @property
     def torch_dtype(self) -> torch.dtype:
@@ -100,6 +124,7 @@ class PoetxLinear:
             xg = torch.empty((T, self.m), dtype=self.torch_dtype, device=self.device)
         if not (save and save_xg):
             xg = None
+        self._dequantize(stream)
         L = self.abi()
         nb = poetx_forward_workspace_bytes(L, T)
         ws = self.workspace("fwd", nb)
@@ -110,8 +135,11 @@ class PoetxLinear:
                  dx: Optional[torch.Tensor] = None, dqR: Optional[torch.Tensor] = None,
                  dqP: Optional[torch.Tensor] = None, accumulate: bool = False, stream=None):
         """dx, dqR, dqP of L = <dz, z>.  `saved` is what forward returned (or
-        just the saved Y tensor)."""
-        if isinstance(saved, torch.Tensor):
+        just the saved Y tensor); None recomputes Y from x (the "mem" variant,
+        which keeps no [T][n] activation between forward and backward)."""
+        if saved is None:
+            saved = Saved(None, None)
+        elif isinstance(saved, torch.Tensor):
             saved = Saved(saved, None)
         T = dz.shape[0]
         if need_dx and dx is None:
@@ -120,8 +148,9 @@ class PoetxLinear:
             dqR = torch.empty_like(self.qR)
         if dqP is None:
             dqP = torch.empty_like(self.qP)
+        self._dequantize(stream)
         L = self.abi()
-        nb = poetx_backward_workspace_bytes(L, T)
+        nb = (poetx_backward_workspace_bytes if saved.y is not None else poetx_backward_recompute_workspace_bytes)(L, T)
         ws = self.workspace("bwd", nb)
         poetx_backward(L, T, x, saved.y, saved.xg, dz, dx if need_dx else None, dqR, dqP, int(accumulate), ws, nb,
                        stream)
@@ -144,11 +173,46 @@ class PoetxLinear:
 
 class LayerGroup:
     """Several layers with the same b and dtype whose G blocks are rebuilt
-    together (one batched CNP build for all of them)."""
+    together (one batched CNP build for all of them), optionally with their
+    packed triangles in one flat buffer (qR then qP of each layer, in order)
+    so one optimizer launch updates all of them."""
 
     def __init__(self, layers):
         self.layers = list(layers)
         self._ws = None
+        self.q = None
+        self.m1 = None
+        self.m2 = None
+        self.steps = 0
+
+    def flatten_params(self) -> torch.Tensor:
+        """Move every layer's qR, qP into one flat fp32 buffer (the layers keep
+        views into it) and allocate the optimizer moments; returns the buffer."""
+        total = sum(L.qR.numel() + L.qP.numel() for L in self.layers)
+        dev = self.layers[0].device
+        self.q = torch.empty(total, dtype=torch.float32, device=dev)
+        off = 0
+        for L in self.layers:
+            for name in ("qR", "qP"):
+                t = getattr(L, name)
+                view = self.q[off:off + t.numel()].view_as(t)
+                view.copy_(t)
+                setattr(L, name, view)
+                off += t.numel()
+        self.m1 = torch.zeros_like(self.q)
+        self.m2 = torch.zeros_like(self.q)
+        return self.q
+
+    def optimizer_step(self, grad: torch.Tensor, lr: float, beta1: float = 0.9, beta2: float = 0.95,
+                       eps: float = 1e-8, weight_decay: float = 0.0, stream=None) -> None:
+        """AdamW on the flat packed triangles with the flat gradient `grad`
+        (same layout), then the batched CNP rebuild of every G."""
+        if self.q is None:
+            raise RuntimeError("flatten_params() first")
+        self.steps += 1
+        poetx_adamw_step(self.q.numel(), self.q, grad, self.m1, self.m2, lr, beta1, beta2, eps, weight_decay,
+                         self.steps, stream)
+        self.build(stream)
 
     def build(self, stream=None) -> None:
         abis = [L.abi() for L in self.layers]

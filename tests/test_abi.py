@@ -81,8 +81,12 @@ def test_validation_before_any_launch(lib):
     assert lib.poetx_forward(ctypes.byref(L), -1, 4096, 4096, None, None, 4096, 1 << 30, None) == 1  # T < 0
     assert lib.poetx_forward(ctypes.byref(L), 10, 4096, 4096, None, None, 4096, 16, None) == 5       # ws small
     assert lib.poetx_forward(ctypes.byref(L), 10, None, 4096, None, None, 4096, 1 << 30, None) == 1  # x NULL
-    assert lib.poetx_backward(ctypes.byref(L), 10, 4096, None, None, 4096, None, 4096, 4096, 0, 4096, 1 << 30,
-                              None) == 1                                                      # y_save NULL
+    assert lib.poetx_backward(ctypes.byref(L), 10, 4096, 4100, None, 4096, None, 4096, 4096, 0, 4096, 1 << 30,
+                              None) == 4                                                      # y_save unaligned
+    # y_save == NULL selects the recomputing backward, which needs a larger workspace
+    assert lib.poetx_backward(ctypes.byref(L), 10, 4096, None, None, 4096, None, 4096, 4096, 0, 4096,
+                              px.poetx_backward_workspace_bytes(L, 10), None) == 5
+    assert px.poetx_backward_recompute_workspace_bytes(L, 10) > px.poetx_backward_workspace_bytes(L, 10)
     assert lib.poetx_backward(ctypes.byref(L), 10, None, 4096, None, 4096, None, 4096, 4096, 0, 4096, 1 << 30,
                               None) == 1                                                      # no x, no xg
     assert lib.poetx_cnp_build(4, 48, 4096, px.POETX_BF16, 4096, 4096, 1 << 30, None) == 2    # b % 64

@@ -232,6 +232,93 @@ def test_saved_xg_backward_matches_regather(case):
         assert np.array_equal(bits(a), bits(b))
 
 
+@pytest.mark.parametrize("case", [("up8b", 512, 1024, 256, 700), ("tiny", 192, 320, 64, 77)], ids=lambda c: c[0])
+def test_recomputing_backward_mem_variant(case):
+    # the "mem" variant keeps nothing from the forward: the backward recomputes
+    # Y from x and must match the saved-Y backward bit for bit
+    inp = _inputs(*case)
+    L = make_layer(inp)
+    x, dz = dev(inp.x, inp.dtype), dev(inp.dz, inp.dtype)
+    _, saved = L.forward(x)
+    dx1, r1, p1 = L.backward(x, saved, dz)
+    dx2, r2, p2 = L.backward(x, None, dz)
+    torch.cuda.synchronize()
+    for a, b in ((dx1, dx2), (r1, r2), (p1, p2)):
+        assert np.array_equal(bits(a), bits(b))
+    _, dxo, dqRo, dqPo, _, _ = _oracle_all(inp)
+    check(host64(dx2), dxo, inp.dtype, "dx (mem variant)")
+    check(host64(r2), dqRo, inp.dtype, "dqR (mem variant)")
+    check(host64(p2), dqPo, inp.dtype, "dqP (mem variant)")
+
+
+@pytest.mark.parametrize("name,m,n,b,T", [("up8b", 512, 768, 256, 300), ("tiny", 192, 320, 64, 77)],
+                         ids=["bf16", "fp32"])
+def test_xq_weight_quantization_and_layer_parity(name, m, n, b, T):
+    # POET-XQ: codes and scales bit-exact against the oracle (both decide them
+    # in float32), the dequantized weight bit-exact, and the layer run on the
+    # dequantized weight against the oracle run on the same weight
+    inp = _inputs(name, m, n, b, T)
+    L = make_layer(inp)
+    stored = host64(L.W)                      # exact stored (frame) weight values
+    L.quantize_weight()
+    z, saved = L.forward(dev(inp.x, inp.dtype))
+    dx, dqR, dqP = L.backward(dev(inp.x, inp.dtype), saved, dev(inp.dz, inp.dtype))
+    torch.cuda.synchronize()
+    codes, scale = oracle.quantize_rows(stored)
+    assert np.array_equal(L.Wq.cpu().numpy(), codes)
+    assert np.array_equal(L.Wscale.cpu().numpy().view(np.uint32), scale.view(np.uint32))
+    deq = oracle.dequantize_rows(codes, scale)
+    want = oracle.round_to_bf16(deq) if inp.dtype == "bf16" else deq.astype(np.float64)
+    assert np.array_equal(host64(L.W), want)
+    W0 = oracle.from_frame(want, inp.permR, inp.permP).T
+    GR, GP = oracle.cnp_blocks(inp.qR, inp.b), oracle.cnp_blocks(inp.qP, inp.b)
+    check(host64(z), oracle.forward(inp.x64, W0, inp.permR, GR, inp.permP, GP), inp.dtype, "z (XQ)")
+    dxo, dqRo, dqPo = oracle.layer_backward(inp.x64, W0, inp.permR, inp.qR, inp.permP, inp.qP, inp.b, inp.dz64)
+    check(host64(dx), dxo, inp.dtype, "dx (XQ)")
+    check(host64(dqR), dqRo, inp.dtype, "dqR (XQ)")
+    check(host64(dqP), dqPo, inp.dtype, "dqP (XQ)")
+
+
+def test_adamw_step_parity():
+    g = np.random.Generator(np.random.PCG64(77))
+    n = 10007                                  # not a multiple of 4: vector body + scalar tail
+    q = (g.standard_normal(n) * 0.01).astype(np.float32)
+    qd, md, vd = torch.from_numpy(q.copy()).cuda(), torch.zeros(n, device="cuda"), torch.zeros(n, device="cuda")
+    qo, mo, vo = q.astype(np.float64), np.zeros(n), np.zeros(n)
+    for step in range(1, 4):
+        grad = g.standard_normal(n).astype(np.float32)
+        px.poetx_adamw_step(n, qd, torch.from_numpy(grad).cuda(), md, vd, 1e-3, 0.9, 0.95, 1e-8, 0.1, step)
+        qo, mo, vo = oracle.adamw_step(qo, grad, mo, vo, 1e-3, 0.9, 0.95, 1e-8, 0.1, step)
+    torch.cuda.synchronize()
+    check(host64(qd), qo, "fp32", "q after 3 AdamW steps")
+    check(host64(md), mo, "fp32", "first moment")
+    check(host64(vd), vo, "fp32", "second moment")
+
+
+def test_fused_optimizer_step_and_rebuild():
+    # AdamW on the flattened packed triangles of two layers, then the batched
+    # CNP rebuild: q and G of each layer against the oracle
+    inps = [_inputs("block8b", 512, 256, 256, 8, layer=0), _inputs("block8b", 256, 768, 256, 8, layer=1)]
+    Ls = [make_layer(i) for i in inps]
+    grp = px.LayerGroup(Ls)
+    flat_q = grp.flatten_params()
+    g = np.random.Generator(np.random.PCG64(5))
+    grads = (g.standard_normal(flat_q.numel()) * 1e-2).astype(np.float32)
+    grp.optimizer_step(torch.from_numpy(grads).cuda(), 1e-3, weight_decay=0.01)
+    torch.cuda.synchronize()
+    off = 0
+    for L, inp in zip(Ls, inps):
+        for name, q0 in (("qR", inp.qR), ("qP", inp.qP)):
+            k = q0.size
+            qo, _, _ = oracle.adamw_step(q0.ravel(), grads[off:off + k], np.zeros(k), np.zeros(k), 1e-3, 0.9, 0.95,
+                                         1e-8, 0.01, 1)
+            off += k
+            q_gpu = getattr(L, name)
+            check(host64(q_gpu).ravel(), qo, "fp32", f"{name} after the step")
+            G = L.GR if name == "qR" else L.GP
+            check(host64(G), oracle.cnp_blocks(host64(q_gpu), inp.b), "bf16", f"G rebuilt from {name}")
+
+
 def test_backward_is_deterministic_and_accumulates():
     inp = _inputs("up8b", 512, 1024, 256, 700)
     L = make_layer(inp)
