@@ -11,7 +11,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libpoetx.so")
 SOURCES = ["poetx.cu"]
-DEPS = ["poetx.cu", "ptx.cuh", "gemm.cuh", "gemm_host.cuh", "perm.cuh", "cnp.cuh", "quant.cuh", "adamw.cuh"]
+DEPS = ["poetx.cu", "ptx.cuh", "gemm.cuh", "gemm_host.cuh", "perm.cuh", "cnp.cuh", "quant.cuh", "adamw.cuh", "gemm2sm.cuh"]
 
 
 def nvcc() -> str:

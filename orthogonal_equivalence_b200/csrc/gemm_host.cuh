@@ -7,6 +7,7 @@
 #include <mutex>
 
 #include "gemm.cuh"
+#include "gemm2sm.cuh"
 
 namespace poetx {
 
@@ -212,9 +213,58 @@ inline cudaError_t launch_simt(const GemmDesc& g, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// The CTA-pair kernel takes plain bf16 products with one batch, no split,
+// K-major A, N a multiple of 256 and a TMA-store output view (the W0 GEMMs).
+inline bool pair_eligible(const GemmDesc& g) {
+  return g.A.et == ET_BF16 && g.B.et == ET_BF16 && !g.A.mn_major && g.batch == 1 && g.splits == 1 &&
+         g.N % tc2::BN == 0 && g.K % tc2::CH == 0 && g.M >= 2 * tc::BM && g.C.et == ET_BF16 &&
+         g.C.view_rows > 0 && g.C.b_row == 0 && g.C.b_col == 0 && !g.add1.ptr && !g.add2.ptr && !g.ex[0].ptr &&
+         !g.ex[1].ptr && !g.C.ptr2 && g.diag == 0.f && (reinterpret_cast<uintptr_t>(g.C.ptr) & 15u) == 0 &&
+         (g.C.ld * 2) % 16 == 0 && g.A.b_row == 0 && g.A.b_col == 0 && g.B.b_row == 0 && g.B.b_col == 0;
+}
+
+inline cudaError_t launch_tc_pair(const GemmDesc& g, cudaStream_t st, int device) {
+  static bool attr_set[64] = {false};
+  if (device >= 0 && device < 64 && !attr_set[device]) {
+    cudaError_t e =
+        cudaFuncSetAttribute(tc2::gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, tc2::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set[device] = true;
+  }
+  CUtensorMap ma, mb, mc;
+  if (!encode_map(&ma, g.A, 128)) return cudaErrorInvalidValue;
+  if (!encode_map(&mb, g.B, g.B.mn_major ? tc2::CH : 128)) return cudaErrorInvalidValue;
+  Operand2D cv;
+  cv.ptr = g.C.ptr;
+  cv.et = ET_BF16;
+  cv.rows = g.C.view_rows;
+  cv.cols = g.C.view_cols;
+  cv.ld = g.C.ld;
+  if (!encode_map(&mc, cv, 32)) return cudaErrorInvalidValue;
+  tc2::Params p;
+  p.M = g.M;
+  p.N = g.N;
+  p.K = g.K;
+  p.tiles_m = (g.M + tc2::BM - 1) / tc2::BM;
+  p.tiles_n = g.N / tc2::BN;
+  p.b_mn = g.B.mn_major;
+  p.idesc = (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(g.B.mn_major) << 16) |
+            (static_cast<uint32_t>(tc2::BN >> 3) << 17) | (static_cast<uint32_t>(tc2::BM >> 4) << 24);
+  p.b_kstep = g.B.mn_major ? tc2::UMMA_K * 128 : 32;
+  p.b_lbo = g.B.mn_major ? tc2::CH * 128 : 16;
+  p.alpha = g.alpha;
+  const int tiles = p.tiles_m * p.tiles_n;
+  const int pairs = sm_count(device) / 2;
+  const int grid = 2 * (tiles < pairs ? tiles : pairs);
+  if (grid <= 0) return cudaSuccess;
+  tc2::gemm_pair_kernel<<<grid, tc2::NUM_THREADS, tc2::SMEM_BYTES, st>>>(ma, mb, mc, p);
+  return cudaGetLastError();
+}
+
 // Tensor cores for bf16 and tf32 operands, FFMA for an all-fp32 layer.
 inline cudaError_t launch_gemm(const GemmDesc& g, bool tensor_cores, cudaStream_t st, int device) {
-  return tensor_cores ? launch_tc(g, st, device) : launch_simt(g, st);
+  if (!tensor_cores) return launch_simt(g, st);
+  return pair_eligible(g) ? launch_tc_pair(g, st, device) : launch_tc(g, st, device);
 }
 
 }  // namespace poetx
