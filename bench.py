@@ -37,10 +37,11 @@ import poetx_inputs as pi  # noqa: E402
 METRIC = "POET-X layer fwd+bwd tokens/s (Llama-8B shapes, b=256); % bf16 tensor peak"
 WORKLOAD = "block8b"
 # DRAM bytes (read + write) per launch of the dominant kernel -- the forward
-# W0 GEMM at M = 16384, N = 14336, K = 4096 -- from an ncu capture of that
-# kernel and shape (dram__bytes_read.sum + dram__bytes_write.sum); reset to
-# None whenever the kernel changes until it is captured again.
-W0_GEMM_TRAFFIC_BYTES = None
+# W0 GEMM (CTA-pair kernel) at M = 16384, N = 14336, K = 4096 -- from an ncu
+# capture of that kernel and shape (dram__bytes_read.sum +
+# dram__bytes_write.sum); reset to None whenever the kernel changes until it
+# is captured again.
+W0_GEMM_TRAFFIC_BYTES = 1109613056 + 456707584
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
