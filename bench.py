@@ -5,10 +5,11 @@ Llama-8B decoder block's seven linears (q, k, v, o, gate, up, down; b = 256,
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl poetx|reference]
 
 One step = the G_R, G_P blocks of every linear built from the packed triangles
-(one batched CNP build), the forwards (saving Y and the gathered input), then
-the backwards in reverse order (dx, dqR, dqP); with N > 1 ranks the
-packed gradients of all linears are summed across ranks (NCCL all-reduce, the
-data-parallel exchange).  Each rank processes its own 16384 tokens (weak
+(one batched CNP build), the forwards (saving Y and the gathered input), the
+backwards in reverse order (dx and the token sums dG of both sides), then one
+batched CNP backward from the dG of all linears to their packed dq; with N > 1
+ranks the packed gradients of all linears are summed across ranks (NCCL
+all-reduce, the data-parallel exchange).  Each rank processes its own 16384 tokens (weak
 scaling).  Inputs are synthetic (seeded normal activations / gradients,
 N(0, 0.02^2) weights, N(0, 0.01^2) triangles, seeded permutations), drawn on
 the device; every tensor of the working set is larger than L2.
@@ -183,8 +184,12 @@ def build_block(cfg: pi.Config, device, rank: int):
         dz = torch.randn((cfg.T, n), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
         layers.append({"L": L, "x": x, "dz": dz, "m": m, "n": n})
     group = px.LayerGroup([l["L"] for l in layers])
-    for l in layers:
+    group.flatten_params()
+    dG = group.dG_buffer()
+    for l, (dGR, dGP) in zip(layers, group.dG_views(dG)):
         l["group"] = group
+        l["dGR"], l["dGP"] = dGR, dGP
+    layers[0]["dG"] = dG
     # outputs and saved activations, allocated once
     nq = sum(l["L"].qR.numel() + l["L"].qP.numel() for l in layers)
     flat = torch.zeros(nq, dtype=torch.float32, device=device)
@@ -202,16 +207,34 @@ def build_block(cfg: pi.Config, device, rank: int):
     return layers, flat
 
 
-def run_step(layers, flat) -> None:
-    # G of every linear from its packed triangles (one batched CNP build), then
-    # the forwards, which keep Y and Xg = x[:, permR] for the backward
-    layers[0]["group"].build()
-    for l in layers:
-        L = l["L"]
-        l["saved"] = L.forward(l["x"], save_xg=True, z=l["z"], y=l["y"], xg=l["xg"])[1]
-    for l in reversed(layers):
-        L = l["L"]
-        L.backward(l["x"], l["saved"], l["dz"], dx=l["dx"], dqR=l["dqR"], dqP=l["dqP"])
+def run_step(layers, flat, mem: bool = False, xs=None, dzs=None, ready=None) -> None:
+    """One step: G of every linear from its packed triangles (one batched CNP
+    build); the forwards, which keep Y and Xg = x[:, permR] for the backward
+    (with `mem`, nothing: the backward recomputes Y); the backwards in reverse
+    order down to dx and the token sums dG; one batched CNP backward from the
+    dG of all linears to their packed dq; the data-parallel gradient sum.
+    `xs`, `dzs` replace the resident inputs; `ready(i, kind)` is called before
+    linear i first reads x ("x") or dz ("dz")."""
+    group = layers[0]["group"]
+    group.build()
+    for i, l in enumerate(layers):
+        x = l["x"] if xs is None else xs[i]
+        if ready:
+            ready(i, "x")
+        if mem:
+            l["L"].forward(x, save=False, z=l["z"])
+            l["saved"] = None
+        else:
+            l["saved"] = l["L"].forward(x, save_xg=True, z=l["z"], y=l["y"], xg=l["xg"])[1]
+    for i in reversed(range(len(layers))):
+        l = layers[i]
+        if ready:
+            ready(i, "dz")
+        l["L"].backward_dG(l["x"] if xs is None else xs[i], l["saved"], l["dz"] if dzs is None else dzs[i],
+                           l["dGR"], l["dGP"], dx=l["dx"])
+        if ready:
+            ready(i, "done")
+    group.cnp_backward(layers[0]["dG"], flat)
     allreduce_grads(flat)
 
 
@@ -311,16 +334,16 @@ def bench_poetx(args, cfg: pi.Config) -> dict:
                 for i in reversed(range(len(layers))):
                     dev_dz[k][i].copy_(host_dz[i], non_blocking=True)
                     dz_ready[k][i].record(copy_stream)
-            layers[0]["group"].build()
-            for i, l in enumerate(layers):
-                stream.wait_event(x_ready[k][i])
-                l["saved"] = l["L"].forward(dev_x[k][i], save_xg=True, z=l["z"], y=l["y"], xg=l["xg"])[1]
-            for i in reversed(range(len(layers))):
-                l = layers[i]
-                stream.wait_event(dz_ready[k][i])
-                l["L"].backward(dev_x[k][i], l["saved"], dev_dz[k][i], dx=l["dx"], dqR=l["dqR"], dqP=l["dqP"])
-                consumed[k][i].record(stream)
-            allreduce_grads(flat)
+
+            def ready(i, kind):
+                if kind == "x":
+                    stream.wait_event(x_ready[k][i])
+                elif kind == "dz":
+                    stream.wait_event(dz_ready[k][i])
+                else:
+                    consumed[k][i].record(stream)
+
+            run_step(layers, flat, xs=dev_x[k], dzs=dev_dz[k], ready=ready)
             host_dq.copy_(flat, non_blocking=True)
 
         e2e_step(0)
@@ -357,12 +380,7 @@ def bench_poetx(args, cfg: pi.Config) -> dict:
             return reduce_max(a.elapsed_time(b_), device) / k
 
         def step_mem():
-            layers[0]["group"].build()
-            for l in layers:
-                l["L"].forward(l["x"], save=False, z=l["z"])
-            for l in reversed(layers):
-                l["L"].backward(l["x"], None, l["dz"], dx=l["dx"], dqR=l["dqR"], dqP=l["dqP"])
-            allreduce_grads(flat)
+            run_step(layers, flat, mem=True)
 
         variants = {}
         step_mem()
@@ -370,7 +388,6 @@ def bench_poetx(args, cfg: pi.Config) -> dict:
         variants["mem"] = {"tokens_per_s": world * cfg.T / (ms / 1e3), "ms_per_step": ms,
                            "note": "backward recomputes Y; no [T][n] activation kept"}
         group = layers[0]["group"]
-        group.flatten_params()
         opt = lambda: group.optimizer_step(flat, 1e-4, weight_decay=0.0)  # noqa: E731
         opt()
         ms = timed(opt, args.steps)

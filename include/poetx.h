@@ -172,6 +172,18 @@ poetx_status poetx_backward(const poetx_layer* layer, int64_t T, const void* x, 
                             const void* xg_save, const void* dz, void* dx, float* dqR, float* dqP,
                             int32_t accumulate, void* ws, size_t ws_bytes, void* stream);
 
+/* poetx_backward with the Cayley-Neumann backward left out: instead of the
+ * packed dq it writes the token sums dGR = dL/dG_R [m/b][b][b] and dGP =
+ * dL/dG_P [n/b][b][b] (fp32, 16-byte aligned; overwritten, or added to when
+ * accumulate != 0), the same fixed-order sums poetx_backward feeds its CNP
+ * backward.  The CNP backward is linear in dG and per block, so one
+ * poetx_cnp_backward over the dG of many layers (blocks back to back in the
+ * order of their packed triangles: qR then qP of each layer) gives all their
+ * dq in one batch.  Same arguments, checks and workspace as poetx_backward. */
+poetx_status poetx_backward_dG(const poetx_layer* layer, int64_t T, const void* x, const void* y_save,
+                               const void* xg_save, const void* dz, void* dx, float* dGR, float* dGP,
+                               int32_t accumulate, void* ws, size_t ws_bytes, void* stream);
+
 /* Merge (merge_if_needed in the write-up's API snippet): writes into W_out
  * ([n][m], dtype, must not overlap layer->W) the weight R W0 P expressed in
  * the frame of new_permR [m], new_permP [n] (device), with R and P built from

@@ -62,6 +62,7 @@ SIGNATURES = {
     "poetx_layer_cnp_build": (ctypes.c_int, [_LP, _VP, _SZ, _VP]),
     "poetx_forward": (ctypes.c_int, [_LP, _I64, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "poetx_backward": (ctypes.c_int, [_LP, _I64, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I32, _VP, _SZ, _VP]),
+    "poetx_backward_dG": (ctypes.c_int, [_LP, _I64, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I32, _VP, _SZ, _VP]),
     "poetx_merge": (ctypes.c_int, [_LP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "poetx_check_perm": (ctypes.c_int, [_VP, _I32, _VP, _VP, _SZ, _VP]),
     "poetx_weight_quantize": (ctypes.c_int, [_I32, _I32, _VP, _I32, _VP, _VP, _VP]),
@@ -215,6 +216,13 @@ def poetx_backward(layer: poetx_layer, T: int, x, y_save, xg_save, dz, dx, dqR, 
     _check(lib().poetx_backward(ctypes.byref(layer), T, _ptr(x), _ptr(y_save), _ptr(xg_save), _ptr(dz), _ptr(dx),
                                 _ptr(dqR), _ptr(dqP), accumulate, _ptr(ws), ws_bytes, _stream(stream)),
            "poetx_backward")
+
+
+def poetx_backward_dG(layer: poetx_layer, T: int, x, y_save, xg_save, dz, dx, dGR, dGP, accumulate: int, ws,
+                      ws_bytes: int, stream=None) -> None:
+    _check(lib().poetx_backward_dG(ctypes.byref(layer), T, _ptr(x), _ptr(y_save), _ptr(xg_save), _ptr(dz),
+                                   _ptr(dx), _ptr(dGR), _ptr(dGP), accumulate, _ptr(ws), ws_bytes, _stream(stream)),
+           "poetx_backward_dG")
 
 
 def poetx_merge(layer: poetx_layer, new_permR, new_permP, W_out, ws, ws_bytes: int, stream=None) -> None:

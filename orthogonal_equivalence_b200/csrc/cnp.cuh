@@ -134,8 +134,11 @@ __global__ void split_blocks_kernel(const Segs sg, const uint8_t* __restrict__ a
 }
 
 // dG = sum over token splits of the partial products, in split order, for
-// both sides; writes dG to o1 (and o2 if given) and dG^T to ot.  32 x 32
-// tiles through shared memory: grid (b/32, b/32, nblk), block (32, 8).
+// both sides; writes dG to o1 (and o2 if given) and dG^T to ot.  One block
+// per 32 x 32 tile: thread (x, y) of the (8, 32) block owns row y, columns
+// 4x..4x+3 (16-byte loads and stores); the transpose goes through shared
+// memory with a padded row, conflict-free.  grid (b/32, b/32, nblk).
+// Requires b % 32 == 0 and 16-byte aligned rows.
 __global__ void reduce_transpose_kernel(const float* __restrict__ part0, int splits0, int n0,
                                         const float* __restrict__ part1, int splits1, int n1, int b,
                                         float* __restrict__ o1, int64_t ld1, int64_t bs1, float* __restrict__ o2,
@@ -158,6 +161,44 @@ __global__ void reduce_transpose_kernel(const float* __restrict__ part0, int spl
     off = (t - n0) * bb;
   }
   const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
+  const int x = threadIdx.x, y = threadIdx.y;
+  const int r = r0 + y, c = c0 + 4 * x;
+  const int64_t e = off + static_cast<int64_t>(r) * b + c;
+  float4 acc = *reinterpret_cast<const float4*>(part + e);
+  for (int s = 1; s < splits; ++s) {
+    const float4 v = *reinterpret_cast<const float4*>(part + s * sstride + e);
+    acc.x += v.x;
+    acc.y += v.y;
+    acc.z += v.z;
+    acc.w += v.w;
+  }
+  *reinterpret_cast<float4*>(o1 + t * bs1 + r * ld1 + c) = acc;
+  if (o2) *reinterpret_cast<float4*>(o2 + t * bs2 + r * ld2 + c) = acc;
+  tile[y][4 * x] = acc.x;
+  tile[y][4 * x + 1] = acc.y;
+  tile[y][4 * x + 2] = acc.z;
+  tile[y][4 * x + 3] = acc.w;
+  __syncthreads();
+  // transposed tile: row c0 + y of dG^T holds column c0 + y of dG
+  const float4 tv = make_float4(tile[4 * x][y], tile[4 * x + 1][y], tile[4 * x + 2][y], tile[4 * x + 3][y]);
+  *reinterpret_cast<float4*>(ot + t * bst + static_cast<int64_t>(c0 + y) * ldt + r0 + 4 * x) = tv;
+}
+
+// Same result for any b (scalar, bounds-checked): grid (ceil(b/32),
+// ceil(b/32), nblk), block (32, 8).
+__global__ void reduce_transpose_any_kernel(const float* __restrict__ part0, int splits0, int n0,
+                                            const float* __restrict__ part1, int splits1, int n1, int b,
+                                            float* __restrict__ o1, int64_t ld1, int64_t bs1, float* __restrict__ o2,
+                                            int64_t ld2, int64_t bs2, float* __restrict__ ot, int64_t ldt,
+                                            int64_t bst) {
+  __shared__ float tile[32][33];
+  const int t = blockIdx.z;
+  const int64_t bb = static_cast<int64_t>(b) * b;
+  const float* part = t < n0 ? part0 : part1;
+  const int splits = t < n0 ? splits0 : splits1;
+  const int64_t sstride = static_cast<int64_t>(t < n0 ? n0 : n1) * bb;
+  const int64_t off = (t < n0 ? t : t - n0) * bb;
+  const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
   for (int i = threadIdx.y; i < 32; i += 8) {
     const int r = r0 + i, c = c0 + threadIdx.x;
     if (r < b && c < b) {
@@ -173,6 +214,41 @@ __global__ void reduce_transpose_kernel(const float* __restrict__ part0, int spl
   for (int i = threadIdx.y; i < 32; i += 8) {
     const int r = c0 + i, c = r0 + threadIdx.x;
     if (r < b && c < b) ot[t * bst + r * ldt + c] = tile[threadIdx.x][i];
+  }
+}
+
+// dG (+)= sum over token splits of the partial products, in split order,
+// for two independent arrays (the two sides of a layer): part_k holds
+// splits_k slices of n4_k float4 each, one slice after the other.  16-byte
+// loads and stores, grid-stride over both arrays.
+__global__ void sum_splits2_kernel(const float4* __restrict__ part0, int splits0, int64_t n40,
+                                   float4* __restrict__ out0, const float4* __restrict__ part1, int splits1,
+                                   int64_t n41, float4* __restrict__ out1, int accumulate) {
+  const int64_t total = n40 + n41;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const bool first = i < n40;
+    const float4* part = first ? part0 : part1;
+    float4* out = first ? out0 : out1;
+    const int splits = first ? splits0 : splits1;
+    const int64_t n4 = first ? n40 : n41;
+    const int64_t e = first ? i : i - n40;
+    float4 acc = part[e];
+    for (int s = 1; s < splits; ++s) {
+      const float4 v = part[s * n4 + e];
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    if (accumulate) {
+      const float4 o = out[e];
+      acc.x = o.x + acc.x;
+      acc.y = o.y + acc.y;
+      acc.z = o.z + acc.z;
+      acc.w = o.w + acc.w;
+    }
+    out[e] = acc;
   }
 }
 

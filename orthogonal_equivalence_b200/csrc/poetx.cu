@@ -599,10 +599,18 @@ poetx_status cnp_backward2(int32_t b, int32_t dtype, const float* q0, int n0, co
                                                         b3, b * b3, Y2, b3, b * b3));
   // dG -> X1[:, b:2b], X2[:, 2b:3b];  dG^T -> Y1[:, 0:b]
   {
-    const dim3 grid((b + 31) / 32, (b + 31) / 32, nblk), block(32, 8);
-    PROFILED(ST_CNP_ELEM, st,
-             reduce_transpose_kernel<<<grid, block, 0, st>>>(part0, splits0, n0, part1, splits1, n1, b, X1 + b, b2,
-                                                             b * b2, X2 + 2 * b, b3, b * b3, Y1, b2, b * b2));
+    if (b % 32 == 0) {
+      const dim3 grid(b / 32, b / 32, nblk), block(8, 32);
+      PROFILED(ST_CNP_ELEM, st,
+               reduce_transpose_kernel<<<grid, block, 0, st>>>(part0, splits0, n0, part1, splits1, n1, b, X1 + b,
+                                                               b2, b * b2, X2 + 2 * b, b3, b * b3, Y1, b2, b * b2));
+    } else {
+      const dim3 grid((b + 31) / 32, (b + 31) / 32, nblk), block(32, 8);
+      PROFILED(ST_CNP_ELEM, st,
+               reduce_transpose_any_kernel<<<grid, block, 0, st>>>(part0, splits0, n0, part1, splits1, n1, b,
+                                                                   X1 + b, b2, b * b2, X2 + 2 * b, b3, b * b3, Y1, b2,
+                                                                   b * b2));
+    }
   }
   POETX_CUDA(cudaGetLastError());
   // S = -(A A^T) -> Y1[:, b:2b];  H^T = (S + 2A)^T -> X1[:, 0:b];  2S -> Y2[:, 2b:3b]
@@ -874,21 +882,26 @@ poetx_status poetx_forward(const poetx_layer* layer, int64_t T, const void* x, v
   return POETX_OK;
 }
 
-poetx_status poetx_backward(const poetx_layer* layer, int64_t T, const void* x, const void* y_save,
-                            const void* xg_save, const void* dz, void* dx, float* dqR, float* dqP,
-                            int32_t accumulate, void* ws, size_t ws_bytes, void* stream) {
+// Backward of one layer.  Gradient mode "dq" (dGR == dGP == NULL): the
+// packed dq of both sides through the CNP backward.  Mode "dG" (dqR == dqP
+// == NULL): the token sums dG of both sides, CNP backward left to the caller.
+static poetx_status backward_impl(const poetx_layer* layer, int64_t T, const void* x, const void* y_save,
+                           const void* xg_save, const void* dz, void* dx, float* dqR, float* dqP, float* dGR,
+                           float* dGP, int32_t accumulate, void* ws, size_t ws_bytes, void* stream) {
   POETX_TRY(check_layer(layer));
   if (T < 0) return POETX_E_ARG;
-  POETX_TRY(check_ptr(dqR));
-  POETX_TRY(check_ptr(dqP));
+  const bool dg_mode = dGR != nullptr;
   const poetx_layer& L = *layer;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int nR = L.m / L.b, nP = L.n / L.b;
-  const size_t triR = size_t(nR) * L.b * (L.b - 1) / 2, triP = size_t(nP) * L.b * (L.b - 1) / 2;
+  const size_t outR = dg_mode ? size_t(nR) * L.b * L.b : size_t(nR) * L.b * (L.b - 1) / 2;
+  const size_t outP = dg_mode ? size_t(nP) * L.b * L.b : size_t(nP) * L.b * (L.b - 1) / 2;
+  float* oR = dg_mode ? dGR : dqR;
+  float* oP = dg_mode ? dGP : dqP;
   if (T == 0) {
     if (!accumulate) {
-      POETX_CUDA(cudaMemsetAsync(dqR, 0, sizeof(float) * triR, st));
-      POETX_CUDA(cudaMemsetAsync(dqP, 0, sizeof(float) * triP, st));
+      POETX_CUDA(cudaMemsetAsync(oR, 0, sizeof(float) * outR, st));
+      POETX_CUDA(cudaMemsetAsync(oP, 0, sizeof(float) * outP, st));
     }
     return POETX_OK;
   }
@@ -913,6 +926,9 @@ poetx_status poetx_backward(const poetx_layer* layer, int64_t T, const void* x, 
   void* dU = c.take<uint8_t>(es * T * L.m);
   float* partP = c.take<float>(sizeof(float) * sP * nP * bb);
   float* partR = c.take<float>(sizeof(float) * sR * nR * bb);
+  // dG mode: a single split without accumulation goes straight to dG
+  if (dg_mode && !accumulate && sP == 1) partP = dGP;
+  if (dg_mode && !accumulate && sR == 1) partR = dGR;
 
   if (recompute) {
     // "mem" variant: Y was not kept; recompute it from x (Xg, U = Xg Diag(G_R), Y = U W~)
@@ -989,10 +1005,42 @@ poetx_status poetx_backward(const poetx_layer* layer, int64_t T, const void* x, 
   PROFILED(ST_DG, st, POETX_CUDA(launch_gemm(blockgrad_desc(Xg, dU, et, T, L.m, L.b, sR, partR), tc_path, st, dev)));
   // dx = dXg Psi_R
   if (dx) PROFILED(ST_PERMUTE, st, POETX_CUDA(permute_dt(L.dtype, dXg, dx, T, L.m, L.permR, 1, st, dev)));
+  if (dg_mode) {
+    // dG = fixed-order sum of the token splits (skipped when the GEMM wrote dG)
+    const bool sumP = partP != dGP, sumR = partR != dGR;
+    if (sumP || sumR) {
+      const int64_t n4P = sumP ? int64_t(nP) * int64_t(bb) / 4 : 0;
+      const int64_t n4R = sumR ? int64_t(nR) * int64_t(bb) / 4 : 0;
+      PROFILED(ST_REDUCE, st,
+               sum_splits2_kernel<<<grid_for(n4P + n4R, 256, dev), 256, 0, st>>>(
+                   reinterpret_cast<const float4*>(partP), sP, n4P, reinterpret_cast<float4*>(dGP),
+                   reinterpret_cast<const float4*>(partR), sR, n4R, reinterpret_cast<float4*>(dGR), accumulate));
+      POETX_CUDA(cudaGetLastError());
+    }
+    return POETX_OK;
+  }
   // dq from the dG partial sums of both sides (fixed-order reduction of the
   // token splits inside the CNP backward)
   POETX_TRY(cnp_backward2(L.b, L.dtype, L.qP, nP, partP, sP, dqP, L.qR, nR, partR, sR, dqR, accumulate, c, st, dev));
   return POETX_OK;
+}
+
+poetx_status poetx_backward(const poetx_layer* layer, int64_t T, const void* x, const void* y_save,
+                            const void* xg_save, const void* dz, void* dx, float* dqR, float* dqP,
+                            int32_t accumulate, void* ws, size_t ws_bytes, void* stream) {
+  POETX_TRY(check_ptr(dqR));
+  POETX_TRY(check_ptr(dqP));
+  return backward_impl(layer, T, x, y_save, xg_save, dz, dx, dqR, dqP, nullptr, nullptr, accumulate, ws, ws_bytes,
+                       stream);
+}
+
+poetx_status poetx_backward_dG(const poetx_layer* layer, int64_t T, const void* x, const void* y_save,
+                               const void* xg_save, const void* dz, void* dx, float* dGR, float* dGP,
+                               int32_t accumulate, void* ws, size_t ws_bytes, void* stream) {
+  POETX_TRY(check_ptr(dGR));
+  POETX_TRY(check_ptr(dGP));
+  return backward_impl(layer, T, x, y_save, xg_save, dz, dx, nullptr, nullptr, dGR, dGP, accumulate, ws, ws_bytes,
+                       stream);
 }
 
 poetx_status poetx_merge(const poetx_layer* layer, const int32_t* new_permR, const int32_t* new_permP,

@@ -12,8 +12,9 @@ from typing import NamedTuple, Optional, Tuple
 
 import torch
 
-from . import (POETX_BF16, POETX_FP32, make_layer, poetx_backward, poetx_backward_recompute_workspace_bytes,
-               poetx_backward_workspace_bytes,
+from . import (POETX_BF16, POETX_FP32, make_layer, poetx_backward, poetx_backward_dG,
+               poetx_backward_recompute_workspace_bytes, poetx_backward_workspace_bytes, poetx_cnp_backward,
+               poetx_cnp_workspace_bytes,
                poetx_forward, poetx_forward_workspace_bytes, poetx_frame_export, poetx_frame_import,
                poetx_layer_cnp_build, poetx_layer_cnp_workspace_bytes, poetx_layers_cnp_build,
                poetx_layers_cnp_workspace_bytes, poetx_merge, poetx_merge_workspace_bytes, poetx_weight_dequantize,
@@ -156,6 +157,27 @@ class PoetxLinear:
                        stream)
         return (dx if need_dx else None), dqR, dqP
 
+    def backward_dG(self, x: torch.Tensor, saved, dz: torch.Tensor, dGR: torch.Tensor, dGP: torch.Tensor,
+                    need_dx: bool = True, dx: Optional[torch.Tensor] = None, accumulate: bool = False,
+                    stream=None) -> Optional[torch.Tensor]:
+        """backward() up to the token sums dGR [m/b][b][b], dGP [n/b][b][b]
+        (fp32), without the CNP backward; LayerGroup.cnp_backward turns the dG
+        of all layers into dq in one batch."""
+        if saved is None:
+            saved = Saved(None, None)
+        elif isinstance(saved, torch.Tensor):
+            saved = Saved(saved, None)
+        T = dz.shape[0]
+        if need_dx and dx is None:
+            dx = torch.empty((T, self.m), dtype=self.torch_dtype, device=self.device)
+        self._dequantize(stream)
+        L = self.abi()
+        nb = (poetx_backward_workspace_bytes if saved.y is not None else poetx_backward_recompute_workspace_bytes)(L, T)
+        ws = self.workspace("bwd", nb)
+        poetx_backward_dG(L, T, x, saved.y, saved.xg, dz, dx if need_dx else None, dGR, dGP, int(accumulate), ws, nb,
+                          stream)
+        return dx if need_dx else None
+
     def merge(self, new_permR: torch.Tensor, new_permP: torch.Tensor, stream=None) -> None:
         """W0 <- R W0 P, re-expressed in the frame of the new permutations;
         q = 0 and G = I afterwards."""
@@ -180,6 +202,7 @@ class LayerGroup:
     def __init__(self, layers):
         self.layers = list(layers)
         self._ws = None
+        self._bws = None
         self.q = None
         self.m1 = None
         self.m2 = None
@@ -213,6 +236,34 @@ class LayerGroup:
         poetx_adamw_step(self.q.numel(), self.q, grad, self.m1, self.m2, lr, beta1, beta2, eps, weight_decay,
                          self.steps, stream)
         self.build(stream)
+
+    def dG_buffer(self) -> torch.Tensor:
+        """A flat fp32 buffer [sum of blocks][b][b] for the dG of every layer,
+        blocks in the order of the packed triangles (R then P of each layer)."""
+        b = self.layers[0].b
+        nblk = sum(L.m // b + L.n // b for L in self.layers)
+        return torch.empty((nblk, b, b), dtype=torch.float32, device=self.layers[0].device)
+
+    def dG_views(self, dG: torch.Tensor):
+        """(dGR, dGP) views of each layer into a dG_buffer()."""
+        out, off = [], 0
+        for L in self.layers:
+            nR, nP = L.m // L.b, L.n // L.b
+            out.append((dG[off:off + nR], dG[off + nR:off + nR + nP]))
+            off += nR + nP
+        return out
+
+    def cnp_backward(self, dG: torch.Tensor, dq: torch.Tensor, accumulate: bool = False, stream=None) -> None:
+        """dq (flat, the layout of flatten_params) from the dG of every layer
+        (dG_buffer layout): one batched CNP backward over all blocks."""
+        if self.q is None:
+            raise RuntimeError("flatten_params() first")
+        L0 = self.layers[0]
+        nblk = dG.shape[0]
+        nb = poetx_cnp_workspace_bytes(nblk, L0.b, L0.dtype)
+        if self._bws is None or self._bws.numel() < nb:
+            self._bws = torch.empty(max(nb, 1), dtype=torch.uint8, device=L0.device)
+        poetx_cnp_backward(nblk, L0.b, self.q, dG, dq, int(accumulate), L0.dtype, self._bws, nb, stream)
 
     def build(self, stream=None) -> None:
         abis = [L.abi() for L in self.layers]

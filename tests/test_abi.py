@@ -23,7 +23,7 @@ def lib():
 def header_functions():
     text = open(os.path.join(ROOT, "include", "poetx.h")).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(poetx_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(poetx_[A-Za-z0-9_]+)\s*\(", text)))
 
 
 def test_header_declares_expected_calls():
@@ -89,6 +89,10 @@ def test_validation_before_any_launch(lib):
     assert px.poetx_backward_recompute_workspace_bytes(L, 10) > px.poetx_backward_workspace_bytes(L, 10)
     assert lib.poetx_backward(ctypes.byref(L), 10, None, 4096, None, 4096, None, 4096, 4096, 0, 4096, 1 << 30,
                               None) == 1                                                      # no x, no xg
+    assert lib.poetx_backward_dG(ctypes.byref(L), 10, 4096, 4096, None, 4096, None, None, 4096, 0, 4096,
+                                 1 << 30, None) == 1                                          # dGR NULL
+    assert lib.poetx_backward_dG(ctypes.byref(L), 10, 4096, 4096, None, 4096, None, 4096, 4104, 0, 4096,
+                                 1 << 30, None) == 4                                          # dGP unaligned
     assert lib.poetx_cnp_build(4, 48, 4096, px.POETX_BF16, 4096, 4096, 1 << 30, None) == 2    # b % 64
     assert lib.poetx_cnp_build(4, 64, 4096, 9, 4096, 4096, 1 << 30, None) == 3
     assert lib.poetx_cnp_build(4, 64, 4096, px.POETX_BF16, 4096, 4096, 8, None) == 5

@@ -334,6 +334,65 @@ def test_backward_is_deterministic_and_accumulates():
     np.testing.assert_allclose(host64(acc_R), 2 * host64(a_R), rtol=1e-6, atol=0)
 
 
+@pytest.mark.parametrize("case", [("up8b", 512, 1024, 256, 700), ("tiny", 192, 320, 64, 77),
+                                  ("down13b", 1024, 1536, 512, 300)], ids=lambda c: c[0])
+def test_dG_backward_and_batched_cnp_backward(case):
+    """poetx_backward_dG: the token sums dG of both sides against the oracle's
+    chain rule, and one poetx_cnp_backward over [dGR | dGP] gives the dq of
+    poetx_backward bit for bit (same sums, same per-block arithmetic)."""
+    inp = _inputs(*case)
+    L = make_layer(inp)
+    x, dz = dev(inp.x, inp.dtype), dev(inp.dz, inp.dtype)
+    _, y = L.forward(x)
+    b, nR, nP = inp.b, inp.m // inp.b, inp.n // inp.b
+    dG = torch.full((nR + nP, b, b), float("nan"), dtype=torch.float32, device="cuda")
+    dx_g = L.backward_dG(x, y, dz, dG[:nR], dG[nR:])
+    dx, dqR, dqP = L.backward(x, y, dz)
+    q = torch.cat([L.qR, L.qP])
+    dq = torch.full_like(q, float("nan"))
+    ws = torch.empty(px.poetx_cnp_workspace_bytes(nR + nP, b, L.dtype), dtype=torch.uint8, device="cuda")
+    px.poetx_cnp_backward(nR + nP, b, q, dG, dq, 0, L.dtype, ws, ws.numel())
+    torch.cuda.synchronize()
+    assert np.array_equal(bits(dx_g), bits(dx))
+    assert np.array_equal(bits(dq[:nR]), bits(dqR)) and np.array_equal(bits(dq[nR:]), bits(dqP))
+    GR, GP = oracle.cnp_blocks(inp.qR, b), oracle.cnp_blocks(inp.qP, b)
+    _, dGRo, dGPo = oracle.backward(inp.x64, inp.W0lin64.T, inp.permR, GR, inp.permP, GP, inp.dz64)
+    check(host64(dG[:nR]), dGRo, inp.dtype, "dGR")
+    check(host64(dG[nR:]), dGPo, inp.dtype, "dGP")
+    # accumulate adds the same sums once more: exactly 2 dG
+    acc = dG.clone()
+    L.backward_dG(x, y, dz, acc[:nR], acc[nR:], need_dx=False, accumulate=True)
+    torch.cuda.synchronize()
+    assert np.array_equal(bits(acc), bits(2 * dG))
+
+
+def test_layer_group_batched_cnp_backward():
+    """Several linears: backward_dG of each into one flat dG buffer, then one
+    batched CNP backward into the flat dq, equals each layer's own dq."""
+    shapes = [(512, 256), (256, 768), (1024, 512)]
+    inps = [_inputs("block8b", m, n, 256, 300, layer=i) for i, (m, n) in enumerate(shapes)]
+    layers = [make_layer(inp) for inp in inps]
+    group = px.LayerGroup(layers)
+    q = group.flatten_params()
+    dG = group.dG_buffer()
+    dq = torch.full_like(q, float("nan"))
+    want = []
+    for L, inp, (dGR, dGP) in zip(layers, inps, group.dG_views(dG)):
+        x, dz = dev(inp.x, "bf16"), dev(inp.dz, "bf16")
+        _, y = L.forward(x)
+        L.backward_dG(x, y, dz, dGR, dGP, need_dx=False)
+        _, dqR, dqP = L.backward(x, y, dz, need_dx=False)
+        want += [dqR.flatten(), dqP.flatten()]
+    group.cnp_backward(dG, dq)
+    torch.cuda.synchronize()
+    assert np.array_equal(bits(dq), bits(torch.cat(want)))
+    for L, inp, (dqR, dqP) in zip(layers, inps, [(want[2 * i], want[2 * i + 1]) for i in range(len(layers))]):
+        _, dqRo, dqPo = oracle.layer_backward(inp.x64, inp.W0lin64.T, inp.permR, inp.qR, inp.permP, inp.qP, inp.b,
+                                              inp.dz64)
+        check(host64(dqR).reshape(dqRo.shape), dqRo, "bf16", "dqR")
+        check(host64(dqP).reshape(dqPo.shape), dqPo, "bf16", "dqP")
+
+
 def test_check_perm_and_errors():
     n = 1000
     perm = torch.from_numpy(pi.permutation(5, n)).cuda()
