@@ -252,6 +252,15 @@ __global__ void sum_splits2_kernel(const float4* __restrict__ part0, int splits0
   }
 }
 
+// dst += src, 16-byte elements, grid-stride.
+__global__ void add_f32x4_kernel(float4* __restrict__ dst, const float4* __restrict__ src, int64_t n4) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float4 a = dst[i], b = src[i];
+    dst[i] = make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+  }
+}
+
 // dq[k(i,j)] (+)= dA[i][j] - dA[j][i] for both sides; one block row per
 // (blk, i).
 __global__ void fold_skew2_kernel(const float* __restrict__ dA, int64_t ld, int64_t bs, int n0, int b,

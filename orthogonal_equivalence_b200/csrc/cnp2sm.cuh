@@ -1,0 +1,521 @@
+// Cayley-Neumann build and backward for b = 256 blocks on CTA pairs (POET-X
+// write-up, section 3: G = (I+Q)(I+Q+Q^2+Q^3) from the packed skew Q, and
+// the gradient of the packed triangle).
+//
+// A grid-wide prep kernel first writes, for every block of the batch, Q in
+// bf16 (Qb) and, for the backward, dG in bf16 (Gb) and the part of dq that
+// needs no product, dq = 2 (dG[i][j] - dG[j][i]).  The fused kernel then takes one 256 x 256 block per pair
+// of SMs at a time: the leader CTA issues every product of the block back to
+// back as tcgen05 MMAs with cta_group::2 (bf16 operands, fp32 accumulation),
+// each CTA keeping the accumulator rows of its half (rows 128*rank .. +127)
+// in its own TMEM.  Operands are read with TMA from Qb, Gb and a per-pair
+// slot (S, H, dS, written by the previous epilogue; one slot per pair,
+// reused block after block, so it stays in L2).  A K-major tile of a matrix
+// is its rows and an MN-major tile its columns, so Q^T = -Q and dG^T, dS^T
+// need no copies.
+//
+// Build (S = Q^2 = -Q Q^T, H = 2Q + S, G = I + 2Q + 2S + H S^T):
+//   P1: acc0 = Q Q^T                          E1: S = -acc0, H = S + 2Q
+//   P2: acc1 = H S^T                          E2: G = I + 2Q + 2S + acc1
+// Backward (dS = 2dG + H^T dG + dG S, dA = 2dG + 2 dG S - dS Q - Q dS,
+// dq_k = dA[i][j] - dA[j][i] for k = k(i, j)):
+//   P1: acc0 = Q Q^T                          E1: S = -acc0, H^T = S - 2Q
+//   P2: acc0 = H^T dG,  acc1 = dG S^T         E2: dS = 2dG + acc0 + acc1;
+//                                                 acc1 <- 2 acc1 (TMEM store)
+//   P3: acc1 += dS Q^T + Q^T dS               E3: acc1 (= dA - 2dG) -> smem
+//   F : dq += acc1[i][j] - acc1[j][i]  (the partner's rows through
+//       distributed shared memory; dq staged in shared memory by bulk copies)
+// The additive terms are added in fp32: S from the fp32 accumulator; I and
+// the 2dG of dq exactly (prep).  2Q in H and G and 2dG in dS, which only
+// feed bf16 operands or the bf16 G, use the bf16 copies the epilogue finds
+// in the staged operand tiles (the last four chunks of a phase always sit in
+// stages 0..3 when its epilogue runs).
+//
+//   warp 0: TMA producer (both CTAs; copies signal the leader's barrier) and
+//           the bulk copies of this CTA's half of dq
+//   warp 1: TMEM owner (both CTAs) and MMA issuer (leader only)
+//   warps 2-5: epilogues; all six warps: fold
+// All threads of both CTAs meet at a cluster barrier between phases.  Every
+// mbarrier wait is bounded (ptx.cuh); after a timeout a thread skips the
+// rest of its work but still takes every cluster barrier.  No load uses
+// multicast.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "cnp.cuh"
+#include "gemm2sm.cuh"
+
+namespace poetx {
+namespace cnp2 {
+
+constexpr int BLK = 256;                 // block size this kernel handles
+constexpr int HALF = 128;                // rows per CTA
+constexpr int CH = 64;                   // K per stage (128 bytes of bf16)
+constexpr int UMMA_K = 16;
+constexpr int TILE_BYTES = HALF * 128;   // 128 rows x 64 bf16, or 64 rows x 2 x 64 (MN-major)
+constexpr int STAGE_BYTES = 2 * TILE_BYTES;
+constexpr int STAGES = 4;
+constexpr int RING_BYTES = STAGES * STAGE_BYTES;
+constexpr int DA_LD = BLK + 1;           // padded fp32 row of acc1 in shared memory
+constexpr int DA_SMEM = HALF * DA_LD * 4;
+constexpr int REGION0 = ((RING_BYTES > DA_SMEM ? RING_BYTES : DA_SMEM) + 1023) & ~1023;
+constexpr int64_t TRI = int64_t(BLK) * (BLK - 1) / 2;
+constexpr int DQ_HALF = static_cast<int>(TRI / 2);      // dq entries per CTA
+constexpr int DQ_BYTES = DQ_HALF * 4;                   // 65280, a multiple of 16
+constexpr int NUM_THREADS = 192;
+constexpr int SMEM_BYTES = REGION0 + DQ_BYTES + 256 + 1024;
+constexpr int SKINDS = 3;                // per-pair slot: S, H (H^T in the backward), dS
+enum SlotKind : int { KS = 0, KH, KDS };
+constexpr size_t MAT_BYTES = size_t(BLK) * BLK * 2;
+
+// Operands of one K chunk: A and B are this CTA's rows (K-major) or, with a
+// "C" suffix, this CTA's columns (MN-major) of the named matrices.
+enum Chunk : int { C_QQ = 0, C_H_S, C_H_GC, C_G_S, C_DS_Q, C_QC_DSC };
+
+struct PairSegs {
+  int n;
+  int start[kMaxSegs + 1];
+  const float* q[kMaxSegs];   // packed triangles [blocks][TRI]
+  const float* dG[kMaxSegs];  // backward: dL/dG [blocks][BLK][BLK]
+  void* out[kMaxSegs];        // build: G (bf16); backward: dq (fp32)
+};
+
+struct Params {
+  int nblk;
+  int backward;
+  uint32_t idesc_kk;       // A K-major, B K-major, M = N = 256
+  uint32_t idesc_kmn;      // A K-major, B MN-major
+  uint32_t idesc_mnmn;     // A MN-major, B MN-major
+  __nv_bfloat16* region;   // [Qb: nblk][Gb: nblk (backward)][slots: pairs x SKINDS], BLK x BLK each
+};
+
+__device__ __forceinline__ int pair_seg_of(const PairSegs& sg, int blk) {
+  int s = 0;
+  while (s + 1 < sg.n && blk >= sg.start[s + 1]) ++s;
+  return s;
+}
+
+// Chunks of phase ph (1-based): count and type of chunk c.
+__device__ __forceinline__ int phase_chunks(int backward, int ph) {
+  return (backward && ph >= 2) ? 8 : 4;
+}
+__device__ __forceinline__ int chunk_type(int backward, int ph, int c) {
+  if (ph == 1) return C_QQ;
+  if (!backward) return C_H_S;
+  if (ph == 2) return c < 4 ? C_H_GC : C_G_S;
+  return c < 4 ? C_DS_Q : C_QC_DSC;
+}
+
+// ---------------------------------------------------------------- prep
+// Qb, and for the backward Gb and dq = 2 (dG[i][j] - dG[j][i]), of
+// the 32 x 32 tile pair (I, J), I <= J, of block blockIdx.y; grid (36, nblk),
+// block (32, 8).
+template <bool BWD>
+__global__ void __launch_bounds__(256) prep_kernel(const __grid_constant__ PairSegs sg,
+                                                   __nv_bfloat16* __restrict__ Qb, __nv_bfloat16* __restrict__ Gb) {
+  __shared__ float tq[32][33];
+  __shared__ float g1[32][33];
+  __shared__ float g2[32][33];
+  const int t = blockIdx.y;
+  int I = 0, x = blockIdx.x;
+  while (x >= 8 - I) {
+    x -= 8 - I;
+    ++I;
+  }
+  const int J = I + x;
+  const int s = pair_seg_of(sg, t), lt = t - sg.start[s];
+  const float* q = sg.q[s] + int64_t(lt) * TRI;
+  __nv_bfloat16* Qt = Qb + size_t(t) * BLK * BLK;
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  const float* dG = BWD ? sg.dG[s] + int64_t(lt) * BLK * BLK : nullptr;
+#pragma unroll
+  for (int r = ty; r < 32; r += 8) {
+    const int i = 32 * I + r, j = 32 * J + tx;
+    tq[r][tx] = j > i ? q[tri_index(i, j, BLK)] : 0.f;
+    if (BWD) {
+      g1[r][tx] = dG[i * BLK + j];
+      g2[r][tx] = dG[(32 * J + r) * BLK + 32 * I + tx];
+    }
+  }
+  __syncthreads();
+  float* dq = BWD ? static_cast<float*>(sg.out[s]) + int64_t(lt) * TRI : nullptr;
+#pragma unroll
+  for (int r = ty; r < 32; r += 8) {
+    const int i = 32 * I + r, j = 32 * J + tx;
+    // tile (I, J); for I < J also its mirror (J, I), Q[j][i] = -Q[i][j]
+    const float v = I < J ? tq[r][tx] : (j > i ? tq[r][tx] : (j < i ? -tq[tx][r] : 0.f));
+    Qt[i * BLK + j] = __float2bfloat16_rn(v);
+    if (I < J) Qt[(32 * J + r) * BLK + 32 * I + tx] = __float2bfloat16_rn(-tq[tx][r]);
+    if (BWD) {
+      __nv_bfloat16* Gt = Gb + size_t(t) * BLK * BLK;
+      Gt[i * BLK + j] = __float2bfloat16_rn(g1[r][tx]);
+      if (I < J) Gt[(32 * J + r) * BLK + 32 * I + tx] = __float2bfloat16_rn(g2[r][tx]);
+      if (j > i) {
+        // dG[j][i]: g2 holds tile (J, I), the tile itself when I == J
+        const float gt = I < J ? g2[tx][r] : g1[tx][r];
+        dq[tri_index(i, j, BLK)] = 2.f * (g1[r][tx] - gt);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- fused kernel
+__device__ __forceinline__ void fence_proxy_async_all() { asm volatile("fence.proxy.async;" ::: "memory"); }
+
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ void bulk_store(void* dst, uint32_t src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src), "r"(bytes)
+               : "memory");
+}
+
+// 32 lanes x 32 consecutive 32-bit columns into TMEM (the inverse of
+// tmem_ld_32cols).
+__device__ __forceinline__ void tmem_st_32cols(uint32_t taddr, const float* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+      "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+      "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+      "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+      "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// 32 bf16 of row r, columns c0 .. c0+31 (c0 % 32 == 0), of a K-major operand
+// staged by TMA: the 128-row x 64-column tile with 128-byte swizzle of stage
+// c0/64 (16-byte chunk u of a row sits at chunk u ^ (r % 8)).
+__device__ __forceinline__ void tile_row_bf16x32(uint32_t tile, int r, int c0, float* v) {
+  const uint32_t rowp = tile + r * 128;
+  const int u0 = (c0 & 63) >> 3;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    uint32_t w[4];
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                 : "r"(rowp + (((u0 + u) ^ (r & 7)) << 4)));
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162*>(&w[h]);
+      v[8 * u + 2 * h] = __low2float(b2);
+      v[8 * u + 2 * h + 1] = __high2float(b2);
+    }
+  }
+}
+__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* p, const float* v) {
+  uint4* d = reinterpret_cast<uint4*>(p);
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    uint4 w;
+    w.x = pack_bf16x2(v[8 * u], v[8 * u + 1]);
+    w.y = pack_bf16x2(v[8 * u + 2], v[8 * u + 3]);
+    w.z = pack_bf16x2(v[8 * u + 4], v[8 * u + 5]);
+    w.w = pack_bf16x2(v[8 * u + 6], v[8 * u + 7]);
+    d[u] = w;
+  }
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+    cnp_pair_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmMN,
+                    const __grid_constant__ PairSegs sg, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  float* dAs = reinterpret_cast<float*>(smem);                // acc1 rows after P3 (over the ring)
+  float* dqs = reinterpret_cast<float*>(smem + REGION0);      // this CTA's half of the block's dq
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + REGION0 + DQ_BYTES);
+  // bars: full[STAGES] (leader), empty[STAGES], acc, dq
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 2);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = tc2::cluster_rank();
+  const bool leader = rank == 0;
+  const uint32_t smem_base = smem_u32(smem);
+  auto bar = [&](int i) { return smem_u32(bars + i); };
+  const int FULL = 0, EMPTY = STAGES, ACC = 2 * STAGES, DQ = 2 * STAGES + 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(bar(FULL + s), 1);
+      mbar_init(bar(EMPTY + s), 1);
+    }
+    mbar_init(bar(ACC), 1);
+    mbar_init(bar(DQ), 1);
+    *s_abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
+                 "r"(512)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  tc2::cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int nph = p.backward ? 3 : 2;
+  const int slot0 = (p.backward ? 2 : 1) * p.nblk + pair * SKINDS;  // matrix index of this pair's S
+  auto matp = [&](int m) { return p.region + size_t(m) * BLK * BLK; };
+  // shared-memory addresses of acc1's rows in both CTAs of the pair
+  const uint32_t dA_cl0 = tc2::map_to_rank(smem_base, 0), dA_cl1 = tc2::map_to_rank(smem_base, 1);
+
+  // ring state (the producer and the MMA issuer each keep their own copy),
+  // carried across phases and blocks; every block issues a multiple of
+  // STAGES chunks, so each phase's last four chunks sit in stages 0..3
+  int stage = 0;
+  uint32_t ring_phase = 0;
+  uint32_t acc_phase = 0, dq_phase = 0;
+
+  auto phase_barrier = [&]() {
+    fence_proxy_async_all();
+    tc_fence_before();
+    __syncwarp();
+    tc2::cluster_sync();
+    tc_fence_after();
+  };
+
+  const int quarter = warp & 3;
+  const int lrow = quarter * 32 + lane;           // this thread's row of the CTA's half in the epilogues
+  const int row = int(rank) * HALF + lrow;        // and of the block
+
+  for (int blk = pair; blk < p.nblk; blk += npairs) {
+    const int s = pair_seg_of(sg, blk);
+    const int lt = blk - sg.start[s];
+    const int mQ = blk, mG = p.nblk + blk;
+    float* dq_g = p.backward ? static_cast<float*>(sg.out[s]) + int64_t(lt) * TRI + int64_t(rank) * DQ_HALF
+                             : nullptr;
+
+    if (p.backward && threadIdx.x == 0 && !*s_abort) {
+      // this CTA's half of dq (2 (dG - dG^T) from the prep) into shared memory
+      bulk_wait_read<0>();  // the previous block's store has read the staging buffer
+      mbar_arrive_expect_tx(bar(DQ), DQ_BYTES);
+      bulk_load(smem_u32(dqs), dq_g, DQ_BYTES, bar(DQ));
+    }
+
+    for (int ph = 1; ph <= nph; ++ph) {
+      const int nch = phase_chunks(p.backward, ph);
+      if (warp == 0) {
+        if (lane == 0 && !*s_abort) {
+          // ---------------- TMA producer
+          for (int c = 0; c < nch; ++c) {
+            if (!mbar_wait(bar(EMPTY + stage), ring_phase ^ 1u, DERR_GEMM_WAIT)) {
+              *s_abort = 1;
+              break;
+            }
+            const int type = chunk_type(p.backward, ph, c);
+            const int k = (c & 3) * CH;
+            const uint32_t full_leader = tc2::map_to_rank(bar(FULL + stage), 0);
+            const uint32_t sa = smem_base + stage * STAGE_BYTES, sb = sa + TILE_BYTES;
+            if (leader) mbar_arrive_expect_tx(bar(FULL + stage), type == C_QQ ? 2 * TILE_BYTES : 2 * STAGE_BYTES);
+            // this CTA's rows (K-major) or columns (MN-major, rows k .. k+63) of matrix m
+            auto rows = [&](uint32_t dst, int m) {
+              tc2::tma_load_2d_pair(dst, &tmK, full_leader, k, m * BLK + int(rank) * HALF);
+            };
+            auto cols = [&](uint32_t dst, int m) {
+              tc2::tma_load_2d_pair(dst, &tmMN, full_leader, int(rank) * HALF, m * BLK + k);
+              tc2::tma_load_2d_pair(dst + CH * 128, &tmMN, full_leader, int(rank) * HALF + CH, m * BLK + k);
+            };
+            switch (type) {
+              case C_QQ: rows(sa, mQ); break;
+              case C_H_S: rows(sa, slot0 + KH); rows(sb, slot0 + KS); break;
+              case C_H_GC: rows(sa, slot0 + KH); cols(sb, mG); break;
+              case C_G_S: rows(sa, mG); rows(sb, slot0 + KS); break;
+              case C_DS_Q: rows(sa, slot0 + KDS); rows(sb, mQ); break;
+              default: cols(sa, mQ); cols(sb, slot0 + KDS); break;  // C_QC_DSC
+            }
+            if (++stage == STAGES) { stage = 0; ring_phase ^= 1u; }
+          }
+        }
+      } else if (warp == 1) {
+        if (leader && lane == 0 && !*s_abort) {
+          // ---------------- MMA issuer (leader, for both CTAs)
+          const uint32_t acc0 = tmem_base, acc1 = tmem_base + BLK;
+          bool ok = true;
+          for (int c = 0; c < nch; ++c) {
+            if (!mbar_wait(bar(FULL + stage), ring_phase, DERR_GEMM_WAIT)) {
+              *s_abort = 1;
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const int type = chunk_type(p.backward, ph, c);
+            const uint32_t sa = smem_base + stage * STAGE_BYTES, sb = sa + TILE_BYTES;
+            const bool a_mn = type == C_QC_DSC;
+            const bool b_mn = type == C_H_GC || type == C_QC_DSC;
+            const uint32_t id = a_mn ? p.idesc_mnmn : (b_mn ? p.idesc_kmn : p.idesc_kk);
+#pragma unroll
+            for (int kk = 0; kk < CH / UMMA_K; ++kk) {
+              const uint64_t da = a_mn ? smem_desc_sw128(sa + kk * (UMMA_K * 128), CH * 128, 1024)
+                                       : smem_desc_sw128(sa + kk * 32, 16, 1024);
+              const uint64_t db = type == C_QQ ? da
+                                  : b_mn       ? smem_desc_sw128(sb + kk * (UMMA_K * 128), CH * 128, 1024)
+                                               : smem_desc_sw128(sb + kk * 32, 16, 1024);
+              const uint32_t fresh = ((c & 3) == 0 && kk == 0) ? 0u : 1u;  // 0: overwrite
+              switch (type) {
+                case C_QQ:
+                case C_H_GC: tc2::mma_pair(acc0, da, db, id, fresh); break;
+                case C_H_S:
+                case C_G_S: tc2::mma_pair(acc1, da, db, id, fresh); break;
+                default: tc2::mma_pair(acc1, da, db, id, 1u); break;  // P3 adds to 2 dG S^T
+              }
+            }
+            tc2::commit_pair(bar(EMPTY + stage));
+            if (++stage == STAGES) { stage = 0; ring_phase ^= 1u; }
+          }
+          if (ok) tc2::commit_pair(bar(ACC));
+        }
+      } else {
+        // ---------------- epilogue of phase ph (this CTA's 128 rows)
+        bool ok = !*s_abort && mbar_wait(bar(ACC), acc_phase, DERR_GEMM_WAIT);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) {
+          if (lane == 0) *s_abort = 1;
+        } else {
+          tc_fence_after();
+          const uint32_t t0 = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+          float v0[32], v1[32], w[32];
+          for (int c0 = 0; c0 < BLK; c0 += 32) {
+            const uint32_t tileA = smem_base + (c0 >> 6) * STAGE_BYTES, tileB = tileA + TILE_BYTES;
+            if (ph == 1) {
+              // S = -acc0;  H = S + 2Q (build) or H^T = S - 2Q (backward); Q from P1's A tiles
+              tmem_ld_32cols(t0 + c0, v0);
+              tile_row_bf16x32(tileA, lrow, c0, w);
+              const float sgn = p.backward ? -2.f : 2.f;
+#pragma unroll
+              for (int e = 0; e < 32; ++e) {
+                v0[e] = -v0[e];
+                v1[e] = v0[e] + sgn * w[e];
+              }
+              store_bf16x32(matp(slot0 + KS) + row * BLK + c0, v0);
+              store_bf16x32(matp(slot0 + KH) + row * BLK + c0, v1);
+            } else if (!p.backward) {
+              // G = I + 2Q + 2S + acc1, 2Q = H - S from P2's A (H) and B (S) tiles, S = -acc0
+              tmem_ld_32cols(t0 + c0, v0);
+              tmem_ld_32cols(t0 + BLK + c0, v1);
+              tile_row_bf16x32(tileA, lrow, c0, w);
+              float sb[32];
+              tile_row_bf16x32(tileB, lrow, c0, sb);
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                v1[e] = ((c0 + e == row ? 1.f : 0.f) + (w[e] - sb[e])) + (-2.f * v0[e]) + v1[e];
+              __nv_bfloat16* G = static_cast<__nv_bfloat16*>(sg.out[s]) + int64_t(lt) * BLK * BLK;
+              store_bf16x32(G + row * BLK + c0, v1);
+            } else if (ph == 2) {
+              // dS = 2dG + acc0 + acc1 (a bf16 operand; dG from P2's A tiles); acc1 <- 2 acc1
+              tmem_ld_32cols(t0 + c0, v0);
+              tmem_ld_32cols(t0 + BLK + c0, v1);
+              tile_row_bf16x32(tileA, lrow, c0, w);
+#pragma unroll
+              for (int e = 0; e < 32; ++e) {
+                v0[e] = (2.f * w[e] + v0[e]) + v1[e];
+                v1[e] = 2.f * v1[e];
+              }
+              store_bf16x32(matp(slot0 + KDS) + row * BLK + c0, v0);
+              tmem_st_32cols(t0 + BLK + c0, v1);
+            } else {
+              // acc1 = dA - 2dG for the fold (padded rows: conflict-free transposed reads)
+              tmem_ld_32cols(t0 + BLK + c0, v0);
+              float* d = dAs + lrow * DA_LD + c0;
+#pragma unroll
+              for (int e = 0; e < 32; ++e) d[e] = v0[e];
+            }
+          }
+        }
+      }
+      acc_phase ^= 1u;
+      phase_barrier();
+    }
+
+    if (p.backward) {
+      // ---------------- F: this CTA's half of dq, k in [rank * DQ_HALF, +DQ_HALF)
+      bool ok = !*s_abort && mbar_wait(bar(DQ), dq_phase, DERR_GEMM_WAIT);
+      dq_phase ^= 1u;
+      if (!ok) *s_abort = 1;
+      __syncwarp();
+      if (!*s_abort) {
+        // element e = tid + 192 m of this CTA's range, k = k0 + e; the row of
+        // k advances monotonically with m.  Loads are issued eight elements
+        // (sixteen loads) at a time.
+        const int k0 = int(rank) * DQ_HALF;
+        const int tid = threadIdx.x;
+        int lo = 0, hi = BLK - 2;  // the row i with start(i) <= k0 + tid < start(i + 1)
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (tri_index(mid, mid + 1, BLK) <= k0 + tid) lo = mid;
+          else hi = mid - 1;
+        }
+        int i = lo;
+        int ks = static_cast<int>(tri_index(i, i + 1, BLK)), ke = ks + (BLK - 1 - i);
+        for (int m0 = 0; m0 * NUM_THREADS < DQ_HALF; m0 += 8) {
+          float a[8], b[8];
+          int idx[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int e = tid + NUM_THREADS * (m0 + u);
+            idx[u] = e < DQ_HALF ? e : -1;
+            if (idx[u] < 0) continue;
+            const int k = k0 + e;
+            while (k >= ke) {
+              ++i;
+              ks = ke;
+              ke = ks + (BLK - 1 - i);
+            }
+            const int j = i + 1 + (k - ks);
+            const uint32_t aij = (i < HALF ? dA_cl0 : dA_cl1) + uint32_t((i & (HALF - 1)) * DA_LD + j) * 4u;
+            const uint32_t aji = (j < HALF ? dA_cl0 : dA_cl1) + uint32_t((j & (HALF - 1)) * DA_LD + i) * 4u;
+            a[u] = ld_cluster_f32(aij);
+            b[u] = ld_cluster_f32(aji);
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            if (idx[u] >= 0) dqs[idx[u]] += a[u] - b[u];
+        }
+      }
+      fence_proxy_async_all();
+      __syncthreads();
+      tc2::cluster_sync();  // both CTAs are done reading each other's rows; staging complete
+      if (threadIdx.x == 0 && !*s_abort) {
+        bulk_store(dq_g, smem_u32(dqs), DQ_BYTES);
+        bulk_commit();
+      }
+    }
+  }
+
+  if (threadIdx.x == 0) bulk_wait_all();
+  if (*s_abort && threadIdx.x == 0) {
+    // give copies already issued time to land before the block leaves
+    const uint64_t t0 = global_ns();
+    while (global_ns() - t0 < 100000ull) {
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc2::cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(512) : "memory");
+  }
+  tc2::cluster_sync();
+}
+
+}  // namespace cnp2
+}  // namespace poetx

@@ -19,6 +19,7 @@
 #include "perm.cuh"
 #include "quant.cuh"
 #include "adamw.cuh"
+#include "cnp2sm.cuh"
 
 using namespace poetx;
 
@@ -46,6 +47,7 @@ struct Carver {
     used += al(bytes);
     return p;
   }
+  bool fits(size_t bytes) const { return used + al(bytes) <= cap; }
 };
 
 #define POETX_TRY(expr)                         \
@@ -516,8 +518,98 @@ Segs two_segs(const float* q0, int n0, void* G0, const float* q1, int n1, void* 
 // G of every segment from its packed triangles, all blocks in one batch.
 // Up to two segments write G straight from the GEMM epilogue; more go
 // through a contiguous scratch copy (`gall`, nblk*b*b elements of dtype).
+// ---- fused CNP on CTA pairs (b = 256, bf16 layers): one kernel per batch,
+// every product of a block on tcgen05 with the operands in an L2-resident
+// per-pair slot (cnp2sm.cuh).
+bool use_pair_cnp(int32_t b, int32_t dtype) { return b == cnp2::BLK && dtype == POETX_BF16; }
+
+int cnp_pair_count(int nblk, int device) {
+  const int pairs = sm_count(device) / 2;
+  return nblk < pairs ? nblk : pairs;
+}
+
+size_t cnp_pair_bytes(int nblk, bool backward, bool accumulate, int device) {
+  const int pairs = cnp_pair_count(nblk, device);
+  return al((size_t(nblk) * (backward ? 2 : 1) + size_t(pairs) * cnp2::SKINDS) * cnp2::MAT_BYTES) +
+         (backward && accumulate ? al(sizeof(float) * size_t(nblk) * cnp2::TRI) : 0);
+}
+
+// Prep (bf16 Q, and for the backward bf16 dG and dq = 2 (dG - dG^T)) and the
+// fused kernel.  With `accumulate` the backward writes its dq into a scratch
+// copy and adds that to the caller's dq at the end, so the sum is exactly
+// dq + (the dq a plain call gives).
+cudaError_t launch_cnp_pair(const cnp2::PairSegs& sg_in, int nblk, bool backward, int accumulate, Carver& ws,
+                            cudaStream_t st, int device) {
+  static bool attr_set[64] = {false};
+  if (device >= 0 && device < 64 && !attr_set[device]) {
+    const cudaError_t e = cudaFuncSetAttribute(cnp2::cnp_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               cnp2::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set[device] = true;
+  }
+  const int pairs = cnp_pair_count(nblk, device);
+  if (pairs <= 0) return cudaSuccess;
+  const int nmat = nblk * (backward ? 2 : 1) + pairs * cnp2::SKINDS;
+  __nv_bfloat16* region = ws.take<__nv_bfloat16>(size_t(nmat) * cnp2::MAT_BYTES);
+  cnp2::PairSegs sg = sg_in;
+  float* dq_tmp = nullptr;
+  if (backward && accumulate) {
+    dq_tmp = ws.take<float>(sizeof(float) * size_t(nblk) * cnp2::TRI);
+    for (int i = 0; i < sg.n; ++i) sg.out[i] = dq_tmp + size_t(sg.start[i]) * cnp2::TRI;
+  }
+  Operand2D v;
+  v.ptr = region;
+  v.et = ET_BF16;
+  v.rows = int64_t(nmat) * cnp2::BLK;
+  v.cols = cnp2::BLK;
+  v.ld = cnp2::BLK;
+  CUtensorMap mk, mm;
+  if (!encode_map(&mk, v, cnp2::HALF) || !encode_map(&mm, v, cnp2::CH)) return cudaErrorInvalidValue;
+  const dim3 pgrid(36, nblk), pblock(32, 8);
+  if (backward)
+    cnp2::prep_kernel<true><<<pgrid, pblock, 0, st>>>(sg, region, region + size_t(nblk) * cnp2::BLK * cnp2::BLK);
+  else
+    cnp2::prep_kernel<false><<<pgrid, pblock, 0, st>>>(sg, region, nullptr);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  cnp2::Params p;
+  p.nblk = nblk;
+  p.backward = backward ? 1 : 0;
+  // D fp32, A and B bf16, N = 256 (bits 17-22: N >> 3), M = 256 (bits 24-28: M >> 4);
+  // bit 15: A MN-major, bit 16: B MN-major
+  p.idesc_kk = (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(cnp2::BLK >> 3) << 17) |
+               (static_cast<uint32_t>(cnp2::BLK >> 4) << 24);
+  p.idesc_kmn = p.idesc_kk | (1u << 16);
+  p.idesc_mnmn = p.idesc_kk | (1u << 15) | (1u << 16);
+  p.region = region;
+  cnp2::cnp_pair_kernel<<<2 * pairs, cnp2::NUM_THREADS, cnp2::SMEM_BYTES, st>>>(mk, mm, sg, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || !dq_tmp) return e;
+  for (int i = 0; i < sg.n; ++i) {
+    const int64_t n4 = int64_t(sg.start[i + 1] - sg.start[i]) * cnp2::TRI / 4;
+    if (n4 <= 0) continue;
+    add_f32x4_kernel<<<grid_for(n4, 256, device), 256, 0, st>>>(static_cast<float4*>(sg_in.out[i]),
+                                                               reinterpret_cast<const float4*>(sg.out[i]), n4);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
 poetx_status cnp_build_segs(int32_t b, int32_t dtype, const Segs& sg, Carver& ws, cudaStream_t st, int device) {
   const int nblk = sg.start[sg.n];
+  if (use_pair_cnp(b, dtype) && ws.fits(cnp_pair_bytes(nblk, false, false, device))) {
+    if (nblk == 0) return POETX_OK;
+    cnp2::PairSegs ps{};
+    ps.n = sg.n;
+    for (int i = 0; i <= sg.n; ++i) ps.start[i] = sg.start[i];
+    for (int i = 0; i < sg.n; ++i) {
+      ps.q[i] = sg.q[i];
+      ps.out[i] = sg.G[i];
+    }
+    PROFILED(ST_CNP_GEMM, st, POETX_CUDA(launch_cnp_pair(ps, nblk, false, 0, ws, st, device)));
+    return POETX_OK;
+  }
   const size_t nbb = size_t(nblk) * b * b;
   float* Q = ws.take<float>(sizeof(float) * nbb);
   float* S = ws.take<float>(sizeof(float) * nbb);
@@ -585,6 +677,38 @@ poetx_status cnp_backward2(int32_t b, int32_t dtype, const float* q0, int n0, co
                            int32_t accumulate, Carver& ws, cudaStream_t st, int device) {
   const int nblk = n0 + n1;
   const size_t nbb = size_t(nblk) * b * b;
+  if (use_pair_cnp(b, dtype) &&
+      ws.fits(((splits0 > 1 || splits1 > 1) ? al(sizeof(float) * nbb) : 0) +
+              cnp_pair_bytes(nblk, true, accumulate != 0, device))) {
+    if (nblk == 0) return POETX_OK;
+    const float* dG0 = part0;
+    const float* dG1 = part1;
+    if (splits0 > 1 || splits1 > 1) {
+      // dG = fixed-order sum of the token splits, both sides into one scratch
+      float* sum = ws.take<float>(sizeof(float) * nbb);
+      const int64_t n40 = int64_t(n0) * b * b / 4, n41 = int64_t(n1) * b * b / 4;
+      PROFILED(ST_REDUCE, st,
+               sum_splits2_kernel<<<grid_for(n40 + n41, 256, device), 256, 0, st>>>(
+                   reinterpret_cast<const float4*>(part0), splits0, n40, reinterpret_cast<float4*>(sum),
+                   reinterpret_cast<const float4*>(part1), splits1, n41, reinterpret_cast<float4*>(sum + n40 * 4), 0));
+      POETX_CUDA(cudaGetLastError());
+      dG0 = sum;
+      dG1 = sum + n40 * 4;
+    }
+    cnp2::PairSegs ps{};
+    ps.n = n1 > 0 ? 2 : 1;
+    ps.start[0] = 0;
+    ps.start[1] = n0;
+    ps.start[2] = n0 + n1;
+    ps.q[0] = q0;
+    ps.dG[0] = dG0;
+    ps.out[0] = dq0;
+    ps.q[1] = q1;
+    ps.dG[1] = dG1;
+    ps.out[1] = dq1;
+    PROFILED(ST_CNP_GEMM, st, POETX_CUDA(launch_cnp_pair(ps, nblk, true, accumulate, ws, st, device)));
+    return POETX_OK;
+  }
   const int64_t b2 = 2 * int64_t(b), b3 = 3 * int64_t(b);
   float* X1 = ws.take<float>(sizeof(float) * 2 * nbb);
   float* Y1 = ws.take<float>(sizeof(float) * 2 * nbb);
