@@ -106,7 +106,10 @@ poetx_status poetx_frame_export(const poetx_layer* layer, void* W0lin, void* str
  * q[nblk][b(b-1)/2] (fp32) writes G[nblk][b][b] (dtype) with
  * G = (I+Q)(I+Q+Q^2+Q^3), evaluated as S = Q Q, G = I + 2Q + 2S + (2Q+S) S
  * (every power of Q is built from Q and S = Q^2).  POETX_FP32: fp32 FFMA;
- * POETX_BF16: tf32 tensor cores, fp32 accumulate, G rounded once to bf16. */
+ * POETX_BF16 with b = 256: one block per pair of SMs, every product on
+ * tcgen05 tensor cores (cta_group::2) with bf16 operands and fp32
+ * accumulation, G rounded once to bf16; POETX_BF16 with other b: a chain of
+ * tcgen05 GEMMs with tf32 operands over the whole batch. */
 poetx_status poetx_cnp_build(int32_t nblk, int32_t b, const float* q, int32_t dtype, void* G, void* ws,
                              size_t ws_bytes, void* stream);
 
@@ -144,8 +147,11 @@ poetx_status poetx_layers_cnp_build(int32_t nlayers, const poetx_layer* layers, 
 /* Backward of poetx_cnp_build: given dG = dL/dG [nblk][b][b] (fp32), writes
  * dq = dL/dq [nblk][b(b-1)/2] (fp32), dq_k = dL/dQ[i][j] - dL/dQ[j][i].
  * accumulate != 0 adds to dq instead of overwriting it.  dtype names the
- * layer precision the gradient serves: POETX_FP32 multiplies in fp32 FFMA,
- * POETX_BF16 on tcgen05 tensor cores with tf32 operands (fp32 accumulate). */
+ * layer precision the gradient serves: POETX_FP32 multiplies in fp32 FFMA;
+ * POETX_BF16 on tcgen05 tensor cores with fp32 accumulation, bf16 operands
+ * for b = 256 (one block per pair of SMs; the terms of dq that need no
+ * product, 2 (dG[i][j] - dG[j][i]), are added in fp32) and tf32 operands for
+ * other b.  Results are identical for every nblk and block order. */
 poetx_status poetx_cnp_backward(int32_t nblk, int32_t b, const float* q, const float* dG, float* dq,
                                 int32_t accumulate, int32_t dtype, void* ws, size_t ws_bytes, void* stream);
 
