@@ -231,7 +231,8 @@ poetx_status poetx_adamw_step(int64_t n, float* q, const float* grad, float* m1,
  * poetx_profile_end(), every kernel the library queues is bracketed by a pair
  * of CUDA events on its stream and tagged with its stage (permute,
  * blockdiag_gemm, w0_gemm, dg_gemm, cnp_gemm, cnp_elementwise, dg_reduce,
- * merge, dequant, optimizer).  poetx_profile_end waits for the recorded events, writes the summed
+ * merge, dequant, optimizer, blockdiag_dg: the backward's block product and
+ * dG partials in one kernel).  poetx_profile_end waits for the recorded events, writes the summed
  * device time in ms (HOST array ms_per_stage[nstages]) and the number of
  * launches (HOST array launches_per_stage[nstages]) per stage, and stops
  * recording.  The events are created on first use and reused. */

@@ -20,6 +20,7 @@
 #include "quant.cuh"
 #include "adamw.cuh"
 #include "cnp2sm.cuh"
+#include "bdg2sm.cuh"
 
 using namespace poetx;
 
@@ -122,10 +123,12 @@ enum Stage : int {
   ST_MERGE,
   ST_DEQUANT,
   ST_OPTIM,
+  ST_BDG,
   ST_COUNT
 };
 const char* const kStageNames[ST_COUNT] = {"permute",  "blockdiag_gemm",  "w0_gemm",   "dg_gemm", "cnp_gemm",
-                                           "cnp_elementwise", "dg_reduce", "merge", "dequant", "optimizer"};
+                                           "cnp_elementwise", "dg_reduce", "merge", "dequant", "optimizer",
+                                            "blockdiag_dg"};
 
 struct Profiler {
   std::mutex mu;
@@ -594,6 +597,56 @@ cudaError_t launch_cnp_pair(const cnp2::PairSegs& sg_in, int nblk, bool backward
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
+}
+
+// ---- fused backward of one side for b = 256 bf16 layers (bdg2sm.cuh):
+// O = D G^T blockwise (skipped when O is NULL) and the split-K partials of
+// dG = X^T D, reading D once.
+bool use_pair_bdg(const poetx_layer& L) { return L.b == bdg2::BLK && L.dtype == POETX_BF16; }
+
+cudaError_t launch_bdg(const void* D, const void* X, const void* G, void* O, float* part, int64_t T, int d, int splits,
+                       cudaStream_t st, int device) {
+  static bool attr_set[64] = {false};
+  if (device >= 0 && device < 64 && !attr_set[device]) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(bdg2::bdg_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bdg2::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set[device] = true;
+  }
+  const int nblk = d / bdg2::BLK;
+  const int ntiles = static_cast<int>((T + bdg2::BLK - 1) / bdg2::BLK);
+  if (splits < 1 || splits > ntiles) return cudaErrorInvalidValue;
+  auto view = [](const void* ptr, int64_t rows, int64_t cols) {
+    Operand2D v;
+    v.ptr = ptr;
+    v.et = ET_BF16;
+    v.rows = rows;
+    v.cols = cols;
+    v.ld = cols;
+    return v;
+  };
+  CUtensorMap mDk, mDmn, mXmn, mG, mO;
+  if (!encode_map(&mDk, view(D, T, d), bdg2::HALF) || !encode_map(&mDmn, view(D, T, d), bdg2::CH) ||
+      !encode_map(&mXmn, view(X, T, d), bdg2::CH) ||
+      !encode_map(&mG, view(G, int64_t(nblk) * bdg2::BLK, bdg2::BLK), bdg2::HALF) ||
+      !encode_map(&mO, view(O ? O : D, T, d), 32))
+    return cudaErrorInvalidValue;
+  bdg2::Params p;
+  p.T = static_cast<int>(T);
+  p.nblk = nblk;
+  p.splits = splits;
+  p.ntiles = ntiles;
+  p.want_o = O ? 1 : 0;
+  // D fp32, A and B bf16, N = 256 (bits 17-22: N >> 3), M = 256 (bits 24-28: M >> 4);
+  // bit 15: A MN-major, bit 16: B MN-major
+  p.idesc_kk = (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(bdg2::BLK >> 3) << 17) |
+               (static_cast<uint32_t>(bdg2::BLK >> 4) << 24);
+  p.idesc_mnmn = p.idesc_kk | (1u << 15) | (1u << 16);
+  p.part = part;
+  const int items = nblk * splits;
+  const int pairs = sm_count(device) / 2 < items ? sm_count(device) / 2 : items;
+  bdg2::bdg_pair_kernel<<<2 * pairs, bdg2::NUM_THREADS, bdg2::SMEM_BYTES, st>>>(mDk, mDmn, mXmn, mG, mO, p);
+  return cudaGetLastError();
 }
 
 poetx_status cnp_build_segs(int32_t b, int32_t dtype, const Segs& sg, Carver& ws, cudaStream_t st, int device) {
@@ -1089,11 +1142,15 @@ static poetx_status backward_impl(const poetx_layer* layer, int64_t T, const voi
   // dV = dz Psi_P^T
   void* dV = bufA;
   PROFILED(ST_PERMUTE, st, POETX_CUDA(permute_dt(L.dtype, dz, dV, T, L.n, L.permP, 0, st, dev)));
-  // dY_j = dV_j G_Pj^T
+  // dY_j = dV_j G_Pj^T and dG_Pj = Y_j^T dV_j (split over tokens): one kernel
+  // reading dV once (b = 256 bf16), else two GEMMs
   void* dY = bufB;
-  PROFILED(ST_BLOCKDIAG, st, POETX_CUDA(launch_gemm(blockdiag_desc(dV, et, T, L.n, L.b, L.GP, true, dY, et), tc_path, st, dev)));
-  // dG_Pj = Y_j^T dV_j (split over tokens)
-  PROFILED(ST_DG, st, POETX_CUDA(launch_gemm(blockgrad_desc(y_save, dV, et, T, L.n, L.b, sP, partP), tc_path, st, dev)));
+  if (use_pair_bdg(L)) {
+    PROFILED(ST_BDG, st, POETX_CUDA(launch_bdg(dV, y_save, L.GP, dY, partP, T, L.n, sP, st, dev)));
+  } else {
+    PROFILED(ST_BLOCKDIAG, st, POETX_CUDA(launch_gemm(blockdiag_desc(dV, et, T, L.n, L.b, L.GP, true, dY, et), tc_path, st, dev)));
+    PROFILED(ST_DG, st, POETX_CUDA(launch_gemm(blockgrad_desc(y_save, dV, et, T, L.n, L.b, sP, partP), tc_path, st, dev)));
+  }
   // dU = dY W~^T  (B(k=j', n=i') = W[j'][i'], MN-major)
   {
     GemmDesc g;
@@ -1122,11 +1179,14 @@ static poetx_status backward_impl(const poetx_layer* layer, int64_t T, const voi
     Xg = bufA;
     PROFILED(ST_PERMUTE, st, POETX_CUDA(permute_dt(L.dtype, x, bufA, T, L.m, L.permR, 0, st, dev)));
   }
-  // dXg_j = dU_j G_Rj^T (dY is dead)
+  // dXg_j = dU_j G_Rj^T (dY is dead; only with dx) and dG_Rj = Xg_j^T dU_j
   void* dXg = bufB;
-  if (dx) PROFILED(ST_BLOCKDIAG, st, POETX_CUDA(launch_gemm(blockdiag_desc(dU, et, T, L.m, L.b, L.GR, true, dXg, et), tc_path, st, dev)));
-  // dG_Rj = Xg_j^T dU_j
-  PROFILED(ST_DG, st, POETX_CUDA(launch_gemm(blockgrad_desc(Xg, dU, et, T, L.m, L.b, sR, partR), tc_path, st, dev)));
+  if (use_pair_bdg(L)) {
+    PROFILED(ST_BDG, st, POETX_CUDA(launch_bdg(dU, Xg, L.GR, dx ? dXg : nullptr, partR, T, L.m, sR, st, dev)));
+  } else {
+    if (dx) PROFILED(ST_BLOCKDIAG, st, POETX_CUDA(launch_gemm(blockdiag_desc(dU, et, T, L.m, L.b, L.GR, true, dXg, et), tc_path, st, dev)));
+    PROFILED(ST_DG, st, POETX_CUDA(launch_gemm(blockgrad_desc(Xg, dU, et, T, L.m, L.b, sR, partR), tc_path, st, dev)));
+  }
   // dx = dXg Psi_R
   if (dx) PROFILED(ST_PERMUTE, st, POETX_CUDA(permute_dt(L.dtype, dXg, dx, T, L.m, L.permR, 1, st, dev)));
   if (dg_mode) {

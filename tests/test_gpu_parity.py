@@ -106,6 +106,39 @@ def test_cnp_build_and_backward_parity(dtype, b, nblk):
     check(host64(dq), 2 * dqo, dtype, "dq accumulated")
 
 
+def test_cnp_full_batch_of_the_8b_block():
+    """The 8B block's batched CNP size (320 blocks of b = 256: several blocks
+    per pair of SMs): build and backward on sampled blocks against the oracle,
+    a sub-batch gives the same bits as the full batch, and accumulating adds
+    exactly the plain result."""
+    nblk, b = 320, 256
+    g = np.random.Generator(np.random.PCG64(4242))
+    q = (g.standard_normal((nblk, b * (b - 1) // 2)) * 0.01).astype(np.float32)
+    dG = g.standard_normal((nblk, b, b)).astype(np.float32)
+    qd, dGd = torch.from_numpy(q).cuda(), torch.from_numpy(dG).cuda()
+    G = torch.empty((nblk, b, b), dtype=torch.bfloat16, device="cuda")
+    nb = px.poetx_cnp_workspace_bytes(nblk, b, px.POETX_BF16)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    px.poetx_cnp_build(nblk, b, qd, px.POETX_BF16, G, ws, nb)
+    dq = torch.full_like(qd, float("nan"))
+    px.poetx_cnp_backward(nblk, b, qd, dGd, dq, 0, px.POETX_BF16, ws, nb)
+    # blocks 147..149 alone (one block per pair)
+    sub_q, sub_dG = qd[147:150].contiguous(), dGd[147:150].contiguous()
+    sub_G = torch.empty((3, b, b), dtype=torch.bfloat16, device="cuda")
+    sub_dq = torch.empty_like(sub_q)
+    px.poetx_cnp_build(3, b, sub_q, px.POETX_BF16, sub_G, ws, nb)
+    px.poetx_cnp_backward(3, b, sub_q, sub_dG, sub_dq, 0, px.POETX_BF16, ws, nb)
+    acc = dq.clone()
+    px.poetx_cnp_backward(nblk, b, qd, dGd, acc, 1, px.POETX_BF16, ws, nb)
+    torch.cuda.synchronize()
+    assert np.array_equal(bits(sub_G), bits(G[147:150])) and np.array_equal(bits(sub_dq), bits(dq[147:150]))
+    assert np.array_equal(bits(acc), bits(2 * dq))
+    for t in [0, 1, 73, 74, 147, 148, 221, 295, 319]:
+        check(host64(G[t]), oracle.cnp_blocks(q[t:t + 1], b)[0], "bf16", f"G[{t}]")
+        check(host64(dq[t]), oracle.cnp_backward(q[t:t + 1], b, dG[t:t + 1].astype(np.float64))[0], "bf16",
+              f"dq[{t}]")
+
+
 @pytest.mark.parametrize("name", ["block8b", "tiny"])
 def test_batched_build_of_several_layers(name):
     # one CNP build for the R and P blocks of several layers equals the
