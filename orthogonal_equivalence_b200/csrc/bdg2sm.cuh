@@ -18,8 +18,10 @@
 //         of its 128 feature columns of X and of D (MN-major, 4 chunks of 64
 //         tokens); each CTA keeps its 128 feature rows of dG_j (TMEM columns
 //         256..511), accumulated over every tile of the item.
-// The O epilogue (TMEM -> bf16 -> swizzled smem boxes -> TMA store) of one
-// tile overlaps MMA2 of that tile and the loads of the next; the dG partial
+// The O epilogue reads the tile's accumulator rows into registers and
+// releases TMEM at once (the next tile's MMA1 waits only for that), then
+// stores them (bf16 -> swizzled smem boxes -> TMA store) while MMA2 of the
+// tile and the next tile's loads proceed; the dG partial
 // (fp32) is written once per item.  Out-of-range token rows of the last tile
 // are zero-filled by TMA (no contribution to dG) and clipped by the TMA
 // store.
@@ -253,37 +255,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           tc_fence_after();
           const int row0 = tile * BLK + int(rank) * HALF + quarter * 32;  // token rows of this warp
           const bool rows_in = row0 < p.T;
-#pragma unroll 1
-          for (int c0 = 0; c0 < BLK; c0 += 64) {
-            uint32_t w[32];
+          // the whole 256-column row into registers (bf16 pairs), then release
+          // the accumulator so the next tile's MMA1 can start while this tile
+          // is stored
+          uint32_t w[BLK / 2];
+#pragma unroll
+          for (int c = 0; c < BLK / 32; ++c) {
             float v[32];
-            tmem_ld_32cols(tl + c0, v);
+            tmem_ld_32cols(tl + 32 * c, v);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
-            tmem_ld_32cols(tl + c0 + 32, v);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) w[16 + i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
-            if (!rows_in) continue;
-            if (lane == 0) bulk_wait_read<1>();
-            __syncwarp();
-            const uint32_t box = my_boxes + buf * EPI_BOX;
-            const uint32_t rowp = box + lane * 128;
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(rowp + ((k ^ (lane & 7)) << 4)),
-                           "r"(w[4 * k]), "r"(w[4 * k + 1]), "r"(w[4 * k + 2]), "r"(w[4 * k + 3])
-                           : "memory");
-            fence_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-              tma_store_2d(&tmO, box, j * BLK + c0, row0);
-              bulk_commit();
-            }
-            buf ^= 1;
+            for (int i = 0; i < 16; ++i) w[16 * c + i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
           }
           tc_fence_before();
           __syncwarp();
           if (lane == 0) tc2::remote_arrive(oempty_leader);
+          if (rows_in) {
+#pragma unroll
+            for (int c0 = 0; c0 < BLK / 64; ++c0) {
+              if (lane == 0) bulk_wait_read<1>();
+              __syncwarp();
+              const uint32_t box = my_boxes + buf * EPI_BOX;
+              const uint32_t rowp = box + lane * 128;
+#pragma unroll
+              for (int k = 0; k < 8; ++k)
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(rowp + ((k ^ (lane & 7)) << 4)),
+                             "r"(w[32 * c0 + 4 * k]), "r"(w[32 * c0 + 4 * k + 1]), "r"(w[32 * c0 + 4 * k + 2]),
+                             "r"(w[32 * c0 + 4 * k + 3])
+                             : "memory");
+              fence_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_2d(&tmO, box, j * BLK + 64 * c0, row0);
+                bulk_commit();
+              }
+              buf ^= 1;
+            }
+          }
         }
         if (!ok) break;
       }

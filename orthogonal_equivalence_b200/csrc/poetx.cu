@@ -570,9 +570,11 @@ cudaError_t launch_cnp_pair(const cnp2::PairSegs& sg_in, int nblk, bool backward
   if (!encode_map(&mk, v, cnp2::HALF) || !encode_map(&mm, v, cnp2::CH)) return cudaErrorInvalidValue;
   const dim3 pgrid(36, nblk), pblock(32, 8);
   if (backward)
-    cnp2::prep_kernel<true><<<pgrid, pblock, 0, st>>>(sg, region, region + size_t(nblk) * cnp2::BLK * cnp2::BLK);
+    PROFILED(ST_CNP_ELEM, st,
+             cnp2::prep_kernel<true><<<pgrid, pblock, 0, st>>>(sg, region,
+                                                               region + size_t(nblk) * cnp2::BLK * cnp2::BLK));
   else
-    cnp2::prep_kernel<false><<<pgrid, pblock, 0, st>>>(sg, region, nullptr);
+    PROFILED(ST_CNP_ELEM, st, cnp2::prep_kernel<false><<<pgrid, pblock, 0, st>>>(sg, region, nullptr));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   cnp2::Params p;
@@ -585,14 +587,16 @@ cudaError_t launch_cnp_pair(const cnp2::PairSegs& sg_in, int nblk, bool backward
   p.idesc_kmn = p.idesc_kk | (1u << 16);
   p.idesc_mnmn = p.idesc_kk | (1u << 15) | (1u << 16);
   p.region = region;
-  cnp2::cnp_pair_kernel<<<2 * pairs, cnp2::NUM_THREADS, cnp2::SMEM_BYTES, st>>>(mk, mm, sg, p);
+  PROFILED(ST_CNP_GEMM, st,
+           cnp2::cnp_pair_kernel<<<2 * pairs, cnp2::NUM_THREADS, cnp2::SMEM_BYTES, st>>>(mk, mm, sg, p));
   e = cudaGetLastError();
   if (e != cudaSuccess || !dq_tmp) return e;
   for (int i = 0; i < sg.n; ++i) {
     const int64_t n4 = int64_t(sg.start[i + 1] - sg.start[i]) * cnp2::TRI / 4;
     if (n4 <= 0) continue;
-    add_f32x4_kernel<<<grid_for(n4, 256, device), 256, 0, st>>>(static_cast<float4*>(sg_in.out[i]),
-                                                               reinterpret_cast<const float4*>(sg.out[i]), n4);
+    PROFILED(ST_CNP_ELEM, st,
+             add_f32x4_kernel<<<grid_for(n4, 256, device), 256, 0, st>>>(
+                 static_cast<float4*>(sg_in.out[i]), reinterpret_cast<const float4*>(sg.out[i]), n4));
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -660,7 +664,7 @@ poetx_status cnp_build_segs(int32_t b, int32_t dtype, const Segs& sg, Carver& ws
       ps.q[i] = sg.q[i];
       ps.out[i] = sg.G[i];
     }
-    PROFILED(ST_CNP_GEMM, st, POETX_CUDA(launch_cnp_pair(ps, nblk, false, 0, ws, st, device)));
+    POETX_CUDA(launch_cnp_pair(ps, nblk, false, 0, ws, st, device));
     return POETX_OK;
   }
   const size_t nbb = size_t(nblk) * b * b;
@@ -759,7 +763,7 @@ poetx_status cnp_backward2(int32_t b, int32_t dtype, const float* q0, int n0, co
     ps.q[1] = q1;
     ps.dG[1] = dG1;
     ps.out[1] = dq1;
-    PROFILED(ST_CNP_GEMM, st, POETX_CUDA(launch_cnp_pair(ps, nblk, true, accumulate, ws, st, device)));
+    POETX_CUDA(launch_cnp_pair(ps, nblk, true, accumulate, ws, st, device));
     return POETX_OK;
   }
   const int64_t b2 = 2 * int64_t(b), b3 = 3 * int64_t(b);
