@@ -7,9 +7,11 @@ Llama-8B decoder block's seven linears (q, k, v, o, gate, up, down; b = 256,
 One step = the G_R, G_P blocks of every linear built from the packed triangles
 (one batched CNP build), the forwards (saving Y and the gathered input), the
 backwards in reverse order (dx and the token sums dG of both sides), then one
-batched CNP backward from the dG of all linears to their packed dq; with N > 1
-ranks the packed gradients of all linears are summed across ranks (NCCL
-all-reduce, the data-parallel exchange).  Each rank processes its own 16384 tokens (weak
+batched CNP backward from the dG of all linears to their packed dq.  With N > 1
+ranks each linear's dG is summed across ranks (NCCL all-reduce, the
+data-parallel exchange) as soon as its backward is done, overlapped with the
+next linear's backward; the CNP backward is linear in dG, so this gives the
+summed dq.  Each rank processes its own 16384 tokens (weak
 scaling).  Inputs are synthetic (seeded normal activations / gradients,
 N(0, 0.02^2) weights, N(0, 0.01^2) triangles, seeded permutations), drawn on
 the device; every tensor of the working set is larger than L2.
@@ -85,6 +87,23 @@ def allreduce_grads(flat) -> None:
     import torch.distributed as dist
     if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
         dist.all_reduce(flat, op=dist.ReduceOp.SUM)
+
+
+def allreduce_start(t):
+    """Start summing `t` across data-parallel ranks without waiting (the
+    collective runs on the communication stream while later kernels run);
+    returns a handle for allreduce_finish, or None with a single rank."""
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        return dist.all_reduce(t, op=dist.ReduceOp.SUM, async_op=True)
+    return None
+
+
+def allreduce_finish(handles) -> None:
+    """Make the current stream wait for every started all-reduce."""
+    for h in handles:
+        if h is not None:
+            h.wait()
 
 
 def barrier(device) -> None:
@@ -186,9 +205,12 @@ def build_block(cfg: pi.Config, device, rank: int):
     group = px.LayerGroup([l["L"] for l in layers])
     group.flatten_params()
     dG = group.dG_buffer()
+    off = 0
     for l, (dGR, dGP) in zip(layers, group.dG_views(dG)):
         l["group"] = group
         l["dGR"], l["dGP"] = dGR, dGP
+        l["dG_all"] = dG[off:off + dGR.shape[0] + dGP.shape[0]]  # both sides, contiguous
+        off += dGR.shape[0] + dGP.shape[0]
     layers[0]["dG"] = dG
     # outputs and saved activations, allocated once
     nq = sum(l["L"].qR.numel() + l["L"].qP.numel() for l in layers)
@@ -226,6 +248,7 @@ def run_step(layers, flat, mem: bool = False, xs=None, dzs=None, ready=None) -> 
             l["saved"] = None
         else:
             l["saved"] = l["L"].forward(x, save_xg=True, z=l["z"], y=l["y"], xg=l["xg"])[1]
+    pending = []
     for i in reversed(range(len(layers))):
         l = layers[i]
         if ready:
@@ -234,8 +257,11 @@ def run_step(layers, flat, mem: bool = False, xs=None, dzs=None, ready=None) -> 
                            l["dGR"], l["dGP"], dx=l["dx"])
         if ready:
             ready(i, "done")
+        # the data-parallel exchange: this linear's dG summed across ranks
+        # while the next linear's backward runs (dq is linear in dG)
+        pending.append(allreduce_start(l["dG_all"]))
+    allreduce_finish(pending)
     group.cnp_backward(layers[0]["dG"], flat)
-    allreduce_grads(flat)
 
 
 def bench_poetx(args, cfg: pi.Config) -> dict:

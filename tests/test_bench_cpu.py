@@ -29,6 +29,10 @@ def _worker(rank, world, port, out):
     import bench
     flat = torch.full((17,), float(rank + 1))
     bench.allreduce_grads(flat)
+    # overlapped form: several tensors started back to back, then waited for
+    parts = [torch.full((5,), float(rank + 1)), torch.full((3,), 10.0 * (rank + 1))]
+    bench.allreduce_finish([bench.allreduce_start(t) for t in parts])
+    assert parts[0].tolist() == [3.0] * 5 and parts[1].tolist() == [30.0] * 3
     slowest = bench.reduce_max(10.0 * rank + 1.5, torch.device("cpu"))
     bench.barrier(torch.device("cpu"))
     out.put((rank, flat.tolist(), slowest))
