@@ -68,7 +68,7 @@ __global__ void __launch_bounds__(256) gather_kernel(const Tin* __restrict__ in,
                                                      Tout* __restrict__ out, int64_t ld_out, int64_t rows, int cols,
                                                      const int32_t* __restrict__ colmap,
                                                      const int32_t* __restrict__ rowmap, int rows_per_iter) {
-  extern __shared__ __align__(16) uint8_t sm_raw[];
+  extern __shared__ __align__(128) uint8_t sm_raw[];
   Tin* sm = reinterpret_cast<Tin*>(sm_raw);
   constexpr int VO = 16 / sizeof(Tout);
   const bool vec_out = (cols % VO == 0) && (ld_out % VO == 0) && ((reinterpret_cast<uintptr_t>(out) & 15u) == 0);
@@ -128,7 +128,7 @@ __global__ void __launch_bounds__(256) scatter_kernel(const T* __restrict__ in, 
                                                       int64_t ld_out, int64_t out_rows, int64_t rows, int cols,
                                                       const int32_t* __restrict__ colmap,
                                                       const int32_t* __restrict__ rowmap, int rows_per_iter) {
-  extern __shared__ __align__(16) uint8_t sm_raw[];
+  extern __shared__ __align__(128) uint8_t sm_raw[];
   T* sm = reinterpret_cast<T*>(sm_raw);
   constexpr int V = 16 / sizeof(T);
   const bool vec_in = (cols % V == 0) && (ld_in % V == 0) && ((reinterpret_cast<uintptr_t>(in) & 15u) == 0);
