@@ -160,7 +160,10 @@ poetx_status poetx_cnp_backward(int32_t nblk, int32_t b, const float* q, const f
  * receives Y = (x Psi_R^T Diag(G_R)) W (the P-side input, in the Psi_P
  * frame) for the backward; pass NULL for inference.  xg_save [T][m] (dtype,
  * nullable) receives Xg = x Psi_R^T, which spares the backward a gather of x.
- * Uses layer->GR/GP as last built by poetx_cnp_build.  T = 0 is a no-op. */
+ * Uses layer->GR/GP as last built by poetx_cnp_build.  T = 0 is a no-op.
+ * bf16 layers with T > n apply Diag(G_R) to the weight rows instead of the
+ * token rows (Y = Xg (W Diag(G_R)^T)^T, same product, rounded once at W_R
+ * instead of at U). */
 poetx_status poetx_forward(const poetx_layer* layer, int64_t T, const void* x, void* z, void* y_save,
                            void* xg_save, void* ws, size_t ws_bytes, void* stream);
 

@@ -56,6 +56,11 @@ struct Carver {
     const poetx_status _s = (expr);             \
     if (_s != POETX_OK) return _s;              \
   } while (0)
+#define POETX_CUDA_ERR(expr)                    \
+  do {                                          \
+    const cudaError_t _e = (expr);              \
+    if (_e != cudaSuccess) return _e;           \
+  } while (0)
 #define POETX_CUDA(expr)                        \
   do {                                          \
     if ((expr) != cudaSuccess) {                \
@@ -653,6 +658,56 @@ cudaError_t launch_bdg(const void* D, const void* X, const void* G, void* O, flo
   return cudaGetLastError();
 }
 
+// Y = (Xg Diag(G_R)) W~^T for T token rows.  When T > n the R-side block
+// product is applied to the n rows of the weight instead of the T rows of
+// activations: W_R = W~ Diag(G_R)^T ([n][m], one weight-sized pass), then
+// Y = Xg W_R^T, which skips the [T][m] intermediate U.  `scratch` holds U
+// ([T][m]) or W_R ([n][m], smaller when T > n).  The choice depends only on
+// (layer, T), so a recomputing backward gets the forward's Y bit for bit.
+bool fold_r_into_weight(const poetx_layer& L, int64_t T) { return L.dtype == POETX_BF16 && T > L.n; }
+
+cudaError_t y_from_xg(const poetx_layer& L, int64_t T, const void* Xg, void* Y, void* scratch, cudaStream_t st,
+                      int dev) {
+  const int et = elem_type(L.dtype);
+  const bool tc_path = use_tc(L.dtype);
+  const void* A;
+  const void* Wb;
+  if (fold_r_into_weight(L, T)) {
+    PROFILED(ST_BLOCKDIAG, st,
+             POETX_CUDA_ERR(launch_gemm(blockdiag_desc(L.W, et, L.n, L.m, L.b, L.GR, true, scratch, et), tc_path, st,
+                                        dev)));
+    A = Xg;
+    Wb = scratch;
+  } else {
+    PROFILED(ST_BLOCKDIAG, st,
+             POETX_CUDA_ERR(launch_gemm(blockdiag_desc(Xg, et, T, L.m, L.b, L.GR, false, scratch, et), tc_path, st,
+                                        dev)));
+    A = scratch;
+    Wb = L.W;
+  }
+  // B(k=i', n=j') = W[j'][i'], K-major
+  GemmDesc g;
+  g.M = static_cast<int>(T);
+  g.N = L.n;
+  g.K = L.m;
+  g.A = colblocks_view(A, et, T, L.m, 0);
+  Operand2D b;
+  b.ptr = Wb;
+  b.et = et;
+  b.rows = L.n;
+  b.cols = L.m;
+  b.ld = L.m;
+  b.mn_major = false;
+  g.B = b;
+  g.C.ptr = Y;
+  g.C.et = et;
+  g.C.ld = L.n;
+  g.C.view_rows = T;
+  g.C.view_cols = L.n;
+  PROFILED(ST_W0, st, POETX_CUDA_ERR(launch_gemm(g, tc_path, st, dev)));
+  return cudaSuccess;
+}
+
 poetx_status cnp_build_segs(int32_t b, int32_t dtype, const Segs& sg, Carver& ws, cudaStream_t st, int device) {
   const int nblk = sg.start[sg.n];
   if (use_pair_cnp(b, dtype) && ws.fits(cnp_pair_bytes(nblk, false, false, device))) {
@@ -1032,30 +1087,9 @@ poetx_status poetx_forward(const poetx_layer* layer, int64_t T, const void* x, v
   void* Y = y_save ? y_save : Yw;
   // Xg = x Psi_R^T  (columns gathered into the Psi_R frame)
   PROFILED(ST_PERMUTE, st, POETX_CUDA(permute_dt(L.dtype, x, Xg, T, L.m, L.permR, 0, st, dev)));
-  // U_j = Xg_j G_Rj
-  PROFILED(ST_BLOCKDIAG, st, POETX_CUDA(launch_gemm(blockdiag_desc(Xg, et, T, L.m, L.b, L.GR, false, U, et), tc_path, st, dev)));
-  // Y = U W~  (W~ = Psi_R W0 Psi_P^T stored [n][m]: B(k=i', n=j') = W[j'][i'], K-major)
-  {
-    GemmDesc g;
-    g.M = static_cast<int>(T);
-    g.N = L.n;
-    g.K = L.m;
-    g.A = colblocks_view(U, et, T, L.m, 0);
-    Operand2D b;
-    b.ptr = L.W;
-    b.et = et;
-    b.rows = L.n;
-    b.cols = L.m;
-    b.ld = L.m;
-    b.mn_major = false;
-    g.B = b;
-    g.C.ptr = Y;
-    g.C.et = et;
-    g.C.ld = L.n;
-    g.C.view_rows = T;
-    g.C.view_cols = L.n;
-    PROFILED(ST_W0, st, POETX_CUDA(launch_gemm(g, tc_path, st, dev)));
-  }
+  // Y = (Xg Diag(G_R)) W~^T  (W~ = Psi_R W0 Psi_P^T stored [n][m]); U in `U`, or
+  // the weight with G_R folded in when T > n
+  POETX_CUDA(y_from_xg(L, T, Xg, Y, U, st, dev));
   // V_j = Y_j G_Pj
   PROFILED(ST_BLOCKDIAG, st, POETX_CUDA(launch_gemm(blockdiag_desc(Y, et, T, L.n, L.b, L.GP, false, V, et), tc_path, st, dev)));
   // z = V Psi_P  (columns scattered back to natural order)
@@ -1112,34 +1146,15 @@ static poetx_status backward_impl(const poetx_layer* layer, int64_t T, const voi
   if (dg_mode && !accumulate && sR == 1) partR = dGR;
 
   if (recompute) {
-    // "mem" variant: Y was not kept; recompute it from x (Xg, U = Xg Diag(G_R), Y = U W~)
+    // "mem" variant: Y was not kept; recompute it from x (Xg, then Y as in the forward)
     void* Ybuf = c.take<uint8_t>(es * T * L.n);
     void* Xbuf = c.take<uint8_t>(es * T * L.m);
     if (!xg_save) {
       PROFILED(ST_PERMUTE, st, POETX_CUDA(permute_dt(L.dtype, x, Xbuf, T, L.m, L.permR, 0, st, dev)));
       xg_save = Xbuf;
     }
-    void* U = dU;  // dU is written only later
-    PROFILED(ST_BLOCKDIAG, st, POETX_CUDA(launch_gemm(blockdiag_desc(xg_save, et, T, L.m, L.b, L.GR, false, U, et), tc_path, st, dev)));
-    GemmDesc g;
-    g.M = static_cast<int>(T);
-    g.N = L.n;
-    g.K = L.m;
-    g.A = colblocks_view(U, et, T, L.m, 0);
-    Operand2D b;
-    b.ptr = L.W;
-    b.et = et;
-    b.rows = L.n;
-    b.cols = L.m;
-    b.ld = L.m;
-    b.mn_major = false;
-    g.B = b;
-    g.C.ptr = Ybuf;
-    g.C.et = et;
-    g.C.ld = L.n;
-    g.C.view_rows = T;
-    g.C.view_cols = L.n;
-    PROFILED(ST_W0, st, POETX_CUDA(launch_gemm(g, tc_path, st, dev)));
+    // the forward's Y, by the same arithmetic (dU, written only later, holds U or the folded weight)
+    POETX_CUDA(y_from_xg(L, T, xg_save, Ybuf, dU, st, dev));
     y_save = Ybuf;
   }
 
