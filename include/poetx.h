@@ -176,7 +176,9 @@ poetx_status poetx_forward(const poetx_layer* layer, int64_t T, const void* x, v
  * write-up's section "三种变体", which keeps no [T][n] activation); its
  * workspace is then poetx_backward_recompute_workspace_bytes.  W0 is frozen,
  * so no dW0.  The dq sums over tokens use a fixed split and order
- * (deterministic for a given shape). */
+ * (deterministic for a given shape).  bf16 layers with T > m form
+ * dU = dV (Diag(G_P)^T W) instead of (dV Diag(G_P)^T) W (same product,
+ * rounded once at the folded weight instead of at dY). */
 poetx_status poetx_backward(const poetx_layer* layer, int64_t T, const void* x, const void* y_save,
                             const void* xg_save, const void* dz, void* dx, float* dqR, float* dqP,
                             int32_t accumulate, void* ws, size_t ws_bytes, void* stream);

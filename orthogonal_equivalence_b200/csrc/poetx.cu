@@ -666,6 +666,11 @@ cudaError_t launch_bdg(const void* D, const void* X, const void* G, void* O, flo
 // (layer, T), so a recomputing backward gets the forward's Y bit for bit.
 bool fold_r_into_weight(const poetx_layer& L, int64_t T) { return L.dtype == POETX_BF16 && T > L.n; }
 
+// Backward P side: dU = dV (Diag(G_P)^T W~) instead of (dV Diag(G_P)^T) W~
+// when T > m (the [n][m] folded weight is smaller than the [T][n] dY it
+// replaces, and fits in the dY buffer).
+bool fold_p_into_weight(const poetx_layer& L, int64_t T) { return L.dtype == POETX_BF16 && T > L.m; }
+
 cudaError_t y_from_xg(const poetx_layer& L, int64_t T, const void* Xg, void* Y, void* scratch, cudaStream_t st,
                       int dev) {
   const int et = elem_type(L.dtype);
@@ -1162,23 +1167,61 @@ static poetx_status backward_impl(const poetx_layer* layer, int64_t T, const voi
   void* dV = bufA;
   PROFILED(ST_PERMUTE, st, POETX_CUDA(permute_dt(L.dtype, dz, dV, T, L.n, L.permP, 0, st, dev)));
   // dY_j = dV_j G_Pj^T and dG_Pj = Y_j^T dV_j (split over tokens): one kernel
-  // reading dV once (b = 256 bf16), else two GEMMs
+  // reading dV once (b = 256 bf16), else two GEMMs.  When T > m (bf16) dY is
+  // not formed at all: G_P is folded into the weight (W_P = Diag(G_P)^T W~,
+  // [n][m], one weight-sized pass) and dU = dV W_P below, so only the dG
+  // product reads dV here.
   void* dY = bufB;
-  if (use_pair_bdg(L)) {
+  const bool fold_p = fold_p_into_weight(L, T);
+  if (fold_p) {
+    // W_P[256j + c][i'] = sum_j' G_Pj[j'][c] W~[256j + j'][i'] for every block j
+    GemmDesc g;
+    g.M = L.b;
+    g.N = L.m;
+    g.K = L.b;
+    g.batch = nP;
+    Operand2D a;
+    a.ptr = L.GP;
+    a.et = et;
+    a.rows = int64_t(nP) * L.b;
+    a.cols = L.b;
+    a.ld = L.b;
+    a.mn_major = true;  // A[c][j'] = G_Pj[j'][c]
+    a.b_row = L.b;
+    g.A = a;
+    Operand2D w;
+    w.ptr = L.W;
+    w.et = et;
+    w.rows = L.n;
+    w.cols = L.m;
+    w.ld = L.m;
+    w.mn_major = true;  // B(k = j', n = i') = W~[256j + j'][i']
+    w.b_row = L.b;
+    g.B = w;
+    g.C.ptr = bufB;
+    g.C.et = et;
+    g.C.ld = L.m;
+    g.C.batch_stride = int64_t(L.b) * L.m;
+    g.C.view_rows = L.n;
+    g.C.view_cols = L.m;
+    g.C.b_row = L.b;
+    PROFILED(ST_BLOCKDIAG, st, POETX_CUDA(launch_gemm(g, tc_path, st, dev)));
+    PROFILED(ST_DG, st, POETX_CUDA(launch_gemm(blockgrad_desc(y_save, dV, et, T, L.n, L.b, sP, partP), tc_path, st, dev)));
+  } else if (use_pair_bdg(L)) {
     PROFILED(ST_BDG, st, POETX_CUDA(launch_bdg(dV, y_save, L.GP, dY, partP, T, L.n, sP, st, dev)));
   } else {
     PROFILED(ST_BLOCKDIAG, st, POETX_CUDA(launch_gemm(blockdiag_desc(dV, et, T, L.n, L.b, L.GP, true, dY, et), tc_path, st, dev)));
     PROFILED(ST_DG, st, POETX_CUDA(launch_gemm(blockgrad_desc(y_save, dV, et, T, L.n, L.b, sP, partP), tc_path, st, dev)));
   }
-  // dU = dY W~^T  (B(k=j', n=i') = W[j'][i'], MN-major)
+  // dU = dY W~^T  (B(k=j', n=i') = W[j'][i'], MN-major), or dU = dV W_P
   {
     GemmDesc g;
     g.M = static_cast<int>(T);
     g.N = L.m;
     g.K = L.n;
-    g.A = colblocks_view(dY, et, T, L.n, 0);
+    g.A = colblocks_view(fold_p ? dV : dY, et, T, L.n, 0);
     Operand2D b;
-    b.ptr = L.W;
+    b.ptr = fold_p ? bufB : L.W;
     b.et = et;
     b.rows = L.n;
     b.cols = L.m;
