@@ -43,6 +43,8 @@ SMALL = [
     ("block8b", 256, 768, 256, 1),
     ("block8b", 512, 1024, 256, 1000),   # >= 4 token tiles: block-resident G path
     ("down13b", 1024, 1536, 512, 777),
+    ("down13b", 1024, 512, 512, 2000),   # T > m, n: both weight folds at b = 512
+    ("attn3b", 256, 384, 128, 1000),     # T > m, n: both weight folds at b = 128
 ]
 
 
