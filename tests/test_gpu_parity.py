@@ -267,7 +267,9 @@ def test_saved_xg_backward_matches_regather(case):
         assert np.array_equal(bits(a), bits(b))
 
 
-@pytest.mark.parametrize("case", [("up8b", 512, 1024, 256, 700), ("tiny", 192, 320, 64, 77)], ids=lambda c: c[0])
+@pytest.mark.parametrize("case", [("up8b", 512, 1024, 256, 700), ("tiny", 192, 320, 64, 77),
+                                  ("block8b", 512, 256, 256, 600)],   # T > m, n: both weight folds
+                         ids=lambda c: f"{c[0]}-{c[4]}")
 def test_recomputing_backward_mem_variant(case):
     # the "mem" variant keeps nothing from the forward: the backward recomputes
     # Y from x and must match the saved-Y backward bit for bit
