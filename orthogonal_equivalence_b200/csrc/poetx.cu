@@ -671,6 +671,54 @@ bool fold_r_into_weight(const poetx_layer& L, int64_t T) { return L.dtype == POE
 // replaces, and fits in the dY buffer).
 bool fold_p_into_weight(const poetx_layer& L, int64_t T) { return L.dtype == POETX_BF16 && T > L.m; }
 
+// Wout = Diag(G_P)^T Win over the n/b row blocks of an [n][m] weight:
+// Wout[bj + c][i'] = sum_j' G_Pj[j'][c] Win[bj + j'][i'] (one batched GEMM).
+cudaError_t fold_p_rows(const poetx_layer& L, const void* Win, void* Wout, cudaStream_t st, int dev) {
+  const int et = elem_type(L.dtype);
+  GemmDesc g;
+  g.M = L.b;
+  g.N = L.m;
+  g.K = L.b;
+  g.batch = L.n / L.b;
+  Operand2D a;
+  a.ptr = L.GP;
+  a.et = et;
+  a.rows = L.n;
+  a.cols = L.b;
+  a.ld = L.b;
+  a.mn_major = true;  // A[c][j'] = G_Pj[j'][c]
+  a.b_row = L.b;
+  g.A = a;
+  Operand2D w;
+  w.ptr = Win;
+  w.et = et;
+  w.rows = L.n;
+  w.cols = L.m;
+  w.ld = L.m;
+  w.mn_major = true;  // B(k = j', n = i') = Win[bj + j'][i']
+  w.b_row = L.b;
+  g.B = w;
+  g.C.ptr = Wout;
+  g.C.et = et;
+  g.C.ld = L.m;
+  g.C.batch_stride = int64_t(L.b) * L.m;
+  g.C.view_rows = L.n;
+  g.C.view_cols = L.m;
+  g.C.b_row = L.b;
+  PROFILED(ST_BLOCKDIAG, st, POETX_CUDA_ERR(launch_gemm(g, use_tc(L.dtype), st, dev)));
+  return cudaSuccess;
+}
+
+// With nothing saved (inference, or a backward that recomputes), a forward
+// of T > 6nm / (2m + 4n) rows is cheaper as one GEMM with the whole layer
+// folded into the weight in the natural frames,
+//   z = x W_eff^T,  W_eff = Psi_P^T Diag(G_P)^T W~ Diag(G_R)^T Psi_R,
+// than as gather, block products and scatter over the token rows (three
+// weight-sized passes instead of 2m + 4n activation columns).
+bool weight_centric_forward(const poetx_layer& L, int64_t T) {
+  return L.dtype == POETX_BF16 && T * (2 * int64_t(L.m) + 4 * int64_t(L.n)) > 6 * int64_t(L.n) * L.m;
+}
+
 cudaError_t y_from_xg(const poetx_layer& L, int64_t T, const void* Xg, void* Y, void* scratch, cudaStream_t st,
                       int dev) {
   const int et = elem_type(L.dtype);
@@ -1083,6 +1131,41 @@ poetx_status poetx_forward(const poetx_layer* layer, int64_t T, const void* x, v
   const int et = elem_type(L.dtype);
   const size_t es = dtype_size(L.dtype);
   const bool tc_path = use_tc(L.dtype);
+  if (!y_save && !xg_save && weight_centric_forward(L, T)) {
+    // two [n][m] weights fit in the workspace whenever this path is chosen
+    Carver cw(ws, ws_bytes);
+    if (cw.fits(2 * al(es * size_t(L.n) * L.m))) {
+      void* W1 = cw.take<uint8_t>(es * size_t(L.n) * L.m);
+      void* W2 = cw.take<uint8_t>(es * size_t(L.n) * L.m);
+      // W1 = W~ Diag(G_R)^T, W2 = Diag(G_P)^T W1, W1 = W2 in natural order
+      PROFILED(ST_BLOCKDIAG, st,
+               POETX_CUDA(launch_gemm(blockdiag_desc(L.W, et, L.n, L.m, L.b, L.GR, true, W1, et), tc_path, st, dev)));
+      POETX_CUDA(fold_p_rows(L, W1, W2, st, dev));
+      PROFILED(ST_PERMUTE, st,
+               POETX_CUDA(scatter_dt(L.dtype, W2, L.m, W1, L.m, L.n, L.n, L.m, L.permR, L.permP, st, dev)));
+      // z = x W1^T
+      GemmDesc g;
+      g.M = static_cast<int>(T);
+      g.N = L.n;
+      g.K = L.m;
+      g.A = colblocks_view(x, et, T, L.m, 0);
+      Operand2D b;
+      b.ptr = W1;
+      b.et = et;
+      b.rows = L.n;
+      b.cols = L.m;
+      b.ld = L.m;
+      b.mn_major = false;
+      g.B = b;
+      g.C.ptr = z;
+      g.C.et = et;
+      g.C.ld = L.n;
+      g.C.view_rows = T;
+      g.C.view_cols = L.n;
+      PROFILED(ST_W0, st, POETX_CUDA(launch_gemm(g, tc_path, st, dev)));
+      return POETX_OK;
+    }
+  }
   Carver c(ws, ws_bytes);
   void* Xw = c.take<uint8_t>(es * T * L.m);
   void* Xg = xg_save ? xg_save : Xw;
@@ -1174,38 +1257,7 @@ static poetx_status backward_impl(const poetx_layer* layer, int64_t T, const voi
   void* dY = bufB;
   const bool fold_p = fold_p_into_weight(L, T);
   if (fold_p) {
-    // W_P[256j + c][i'] = sum_j' G_Pj[j'][c] W~[256j + j'][i'] for every block j
-    GemmDesc g;
-    g.M = L.b;
-    g.N = L.m;
-    g.K = L.b;
-    g.batch = nP;
-    Operand2D a;
-    a.ptr = L.GP;
-    a.et = et;
-    a.rows = int64_t(nP) * L.b;
-    a.cols = L.b;
-    a.ld = L.b;
-    a.mn_major = true;  // A[c][j'] = G_Pj[j'][c]
-    a.b_row = L.b;
-    g.A = a;
-    Operand2D w;
-    w.ptr = L.W;
-    w.et = et;
-    w.rows = L.n;
-    w.cols = L.m;
-    w.ld = L.m;
-    w.mn_major = true;  // B(k = j', n = i') = W~[256j + j'][i']
-    w.b_row = L.b;
-    g.B = w;
-    g.C.ptr = bufB;
-    g.C.et = et;
-    g.C.ld = L.m;
-    g.C.batch_stride = int64_t(L.b) * L.m;
-    g.C.view_rows = L.n;
-    g.C.view_cols = L.m;
-    g.C.b_row = L.b;
-    PROFILED(ST_BLOCKDIAG, st, POETX_CUDA(launch_gemm(g, tc_path, st, dev)));
+    POETX_CUDA(fold_p_rows(L, L.W, bufB, st, dev));
     PROFILED(ST_DG, st, POETX_CUDA(launch_gemm(blockgrad_desc(y_save, dV, et, T, L.n, L.b, sP, partP), tc_path, st, dev)));
   } else if (use_pair_bdg(L)) {
     PROFILED(ST_BDG, st, POETX_CUDA(launch_bdg(dV, y_save, L.GP, dY, partP, T, L.n, sP, st, dev)));

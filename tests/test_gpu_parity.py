@@ -267,6 +267,24 @@ def test_saved_xg_backward_matches_regather(case):
         assert np.array_equal(bits(a), bits(b))
 
 
+@pytest.mark.parametrize("case", [("block8b", 512, 256, 256, 2000), ("up8b", 256, 768, 256, 1500),
+                                  ("attn3b", 512, 512, 256, 300)], ids=lambda c: f"{c[0]}-{c[4]}")
+def test_forward_without_saving(case):
+    """A forward that saves nothing (inference, or the recomputing backward's
+    forward): above T = 6nm/(2m+4n) the whole layer is one GEMM with the
+    weight folded into the natural frames; z against the oracle and against
+    the forward that saves Y (which takes the token-row path)."""
+    inp = _inputs(*case)
+    L = make_layer(inp)
+    x = dev(inp.x, inp.dtype)
+    z_nosave, _ = L.forward(x, save=False)
+    z_save, _ = L.forward(x)
+    torch.cuda.synchronize()
+    zo, _, _, _, _, _ = _oracle_all(inp)
+    check(host64(z_nosave), zo, inp.dtype, "z (nothing saved)")
+    check(host64(z_nosave), host64(z_save), inp.dtype, "z (nothing saved vs saved)")
+
+
 @pytest.mark.parametrize("case", [("up8b", 512, 1024, 256, 700), ("tiny", 192, 320, 64, 77),
                                   ("block8b", 512, 256, 256, 600)],   # T > m, n: both weight folds
                          ids=lambda c: f"{c[0]}-{c[4]}")
