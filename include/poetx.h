@@ -163,7 +163,10 @@ poetx_status poetx_cnp_backward(int32_t nblk, int32_t b, const float* q, const f
  * Uses layer->GR/GP as last built by poetx_cnp_build.  T = 0 is a no-op.
  * bf16 layers with T > n apply Diag(G_R) to the weight rows instead of the
  * token rows (Y = Xg (W Diag(G_R)^T)^T, same product, rounded once at W_R
- * instead of at U). */
+ * instead of at U).  With y_save == xg_save == NULL (inference) and
+ * T > 6nm/(2m+4n), bf16 layers fold the whole layer into one natural-frame
+ * weight and compute z = x W_eff^T as a single GEMM (same product, rounded
+ * at the folded weights instead of at the activations). */
 poetx_status poetx_forward(const poetx_layer* layer, int64_t T, const void* x, void* z, void* y_save,
                            void* xg_save, void* ws, size_t ws_bytes, void* stream);
 
