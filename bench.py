@@ -22,6 +22,7 @@ a bounded token sample of the same workload.
 from __future__ import annotations
 
 import argparse
+import datetime
 import json
 import os
 import statistics
@@ -117,9 +118,12 @@ def barrier(device) -> None:
 
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    """nvidia-smi clock / throttle-reason samples around the timed region.
+    Each sample carries nvidia-smi's own timestamp; `mark_begin` / `mark_end`
+    bracket the region on the host clock and only the samples inside it count
+    as "under load" (the median clock, the instantaneous power)."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw.instant,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
     NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
@@ -129,13 +133,21 @@ class ClockSampler:
         self.proc = None
         self.lines = []
         self.thread = None
+        self.t_begin = None
+        self.t_end = None
 
     def start(self):
+        fields = self.FIELDS
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+            # drivers without the instantaneous power field: the averaged one
+            probe = subprocess.run(["nvidia-smi", f"--query-gpu={fields}", "--format=csv,noheader,nounits", "-i",
+                                    self.gpu_id], capture_output=True, text=True, timeout=20)
+            if probe.returncode != 0:
+                fields = fields.replace("power.draw.instant", "power.draw")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={fields}", "--format=csv,noheader,nounits",
                                           "-lms", "50", "-i", self.gpu_id], stdout=subprocess.PIPE,
                                          stderr=subprocess.DEVNULL, text=True)
-        except OSError:
+        except (OSError, subprocess.TimeoutExpired):
             self.proc = None
             return
         self.thread = threading.Thread(target=self._read, daemon=True)
@@ -145,9 +157,59 @@ class ClockSampler:
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
+    def mark_begin(self):
+        self.t_begin = time.time()
+
+    def mark_end(self):
+        self.t_end = time.time()
+
+    @staticmethod
+    def parse(lines, t_begin=None, t_end=None) -> dict:
+        """Samples -> the clocks record.  Samples outside [t_begin, t_end]
+        (when both are given and at least one sample falls inside) are
+        dropped; reasons are collected over the kept samples."""
+        rows = []
+        for ln in lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except ValueError:
+                ts = None
+            try:
+                sm, smax = float(parts[2]), float(parts[3])
+            except ValueError:
+                continue
+            try:
+                power = float(parts[4])
+            except ValueError:
+                power = None
+            rows.append((ts, sm, smax, power, parts[6:10]))
+        inside = rows
+        if t_begin is not None and t_end is not None:
+            sel = [r for r in rows if r[0] is not None and t_begin <= r[0] <= t_end]
+            if sel:
+                inside = sel
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no nvidia-smi samples"], "samples": 0}
+        reasons = set()
+        for r in inside:
+            for name, v in zip(ClockSampler.NAMES, r[4]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        powers = [r[3] for r in inside if r[3] is not None]
+        return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_max_mhz": max(r[2] for r in inside),
+                "reasons": sorted(reasons), "samples": len(inside), "samples_total": len(rows),
+                "sm_mhz_min": min(r[1] for r in inside),
+                "power_w_median": statistics.median(powers) if powers else None,
+                "power_w_max": max(powers) if powers else None,
+                "window": "samples stamped inside the timed region" if inside is not rows else "all samples"}
+
     def stop(self) -> dict:
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.1)  # the sample that covers the region's end
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -155,23 +217,7 @@ class ClockSampler:
             self.proc.kill()
         if self.thread:
             self.thread.join(timeout=5)
-        sm, smax, power, reasons = [], [], [], set()
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax.append(float(parts[2]))
-                power.append(float(parts[3]))
-            except ValueError:
-                continue
-            for name, v in zip(self.NAMES, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(name)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm),
-                "power_w_max": max(power) if power else None}
+        return self.parse(self.lines, self.t_begin, self.t_end)
 
 
 # ---------------------------------------------------------------- POET-X arm
@@ -272,7 +318,6 @@ def bench_poetx(args, cfg: pi.Config) -> dict:
 
     rank, world, local = dist_env()
     if world > 1:
-        import datetime
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     device = torch.device("cuda", local)
@@ -299,11 +344,13 @@ def bench_poetx(args, cfg: pi.Config) -> dict:
     # ends (value, ms_per_step).
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(device)
+    sampler.mark_begin()
     start.record(stream)
     for _ in range(args.steps):
         run_step(layers, flat)
     end.record(stream)
     torch.cuda.synchronize(device)
+    sampler.mark_end()
     barrier(device)
     clocks = sampler.stop()
     ms_local = start.elapsed_time(end)

@@ -85,3 +85,28 @@ def test_bench_rejects_short_warmup():
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--warmup", "2"],
                          capture_output=True, text=True, timeout=120, cwd=ROOT)
     assert out.returncode != 0
+
+
+def test_clock_samples_inside_timed_region():
+    # only samples stamped inside [t_begin, t_end] count as under load
+    import datetime
+    import bench
+
+    def line(sec, mhz, power, cap="Not Active"):
+        ts = datetime.datetime(2026, 1, 1, 12, 0, 0) + datetime.timedelta(seconds=sec)
+        stamp = ts.strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+        return f"{stamp}, 0, {mhz}, 1965, {power}, 0x0, Not Active, Not Active, Not Active, {cap}"
+
+    t0 = datetime.datetime(2026, 1, 1, 12, 0, 0).timestamp()
+    lines = [line(0.0, 1965, 150.0), line(0.1, 1965, 160.0), line(0.5, 1300, 990.0, "Active"),
+             line(0.55, 1320, 1000.0, "Active"), line(0.6, 1310, 980.0), line(1.5, 1965, 200.0)]
+    rec = bench.ClockSampler.parse(lines, t0 + 0.45, t0 + 0.65)
+    assert rec["samples"] == 3 and rec["samples_total"] == 6
+    assert rec["sm_mhz"] == 1310 and rec["sm_mhz_min"] == 1300
+    assert rec["reasons"] == ["sw_power_cap"]
+    assert rec["power_w_max"] == 1000.0
+    # no window given: every sample counts
+    rec = bench.ClockSampler.parse(lines)
+    assert rec["samples"] == 6 and rec["window"] == "all samples"
+    # malformed lines are skipped
+    assert bench.ClockSampler.parse(["garbage", ""])["samples"] == 0
