@@ -64,6 +64,9 @@ def config_block(cfg: pi.Config, n_gpus: int) -> dict:
             "linears": [f"{nm} {m}x{n}" for nm, m, n in cfg.layers],
             "tokens_per_gpu": cfg.T, "global_batch": cfg.T * n_gpus, "seq_len": 2048, "b": cfg.b,
             "parallelism": f"dp{n_gpus}",
+            "shared_inputs": [",".join(cfg.layers[i][0] for i in range(len(cfg.layers)) if cfg.x_source(i) == j)
+                              for j in sorted({cfg.x_source(i) for i in range(len(cfg.layers))})
+                              if sum(cfg.x_source(i) == j for i in range(len(cfg.layers))) > 1],
             "l2": "no flush: every input and intermediate is larger than the 126 MB L2"}
 
 
@@ -242,12 +245,17 @@ def build_block(cfg: pi.Config, device, rank: int):
         L = px.PoetxLinear(m, n, cfg.b, px.POETX_BF16, device=device)
         L.load(W0lin, permR, permP, qR, qP)
         del W0lin
-        # per-rank data (each data-parallel rank sees its own tokens)
-        g.manual_seed(pi.seed_of(cfg, li, "x") + 7919 * rank)
-        x = torch.randn((cfg.T, m), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+        # per-rank data (each data-parallel rank sees its own tokens); linears
+        # of a block that read the same hidden state share one x
+        src = cfg.x_source(li)
+        if src != li:
+            x = layers[src]["x"]
+        else:
+            g.manual_seed(pi.seed_of(cfg, li, "x") + 7919 * rank)
+            x = torch.randn((cfg.T, m), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
         g.manual_seed(pi.seed_of(cfg, li, "dz") + 7919 * rank)
         dz = torch.randn((cfg.T, n), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
-        layers.append({"L": L, "x": x, "dz": dz, "m": m, "n": n})
+        layers.append({"L": L, "x": x, "dz": dz, "m": m, "n": n, "x_src": src})
     group = px.LayerGroup([l["L"] for l in layers])
     group.flatten_params()
     dG = group.dG_buffer()
@@ -374,24 +382,27 @@ def bench_poetx(args, cfg: pi.Config) -> dict:
     barrier(device)
     ms_profiled = reduce_max(p_start.elapsed_time(p_end), device)
 
-    # End to end through the public API: every step copies its inputs (x and
-    # dz of every linear) from pinned host memory and reads the packed
-    # gradients back.  The copies run on their own stream into two alternating
-    # sets of device buffers, so step s+1's inputs stream in while step s
-    # computes; each linear waits only for its own inputs.
+    # End to end through the public API: every step copies its inputs (each
+    # distinct x, which q/k/v and gate/up share, and the dz of every linear)
+    # from pinned host memory and reads the packed gradients back.  The
+    # copies run on their own stream into two alternating sets of device
+    # buffers, so step s+1's inputs stream in while step s computes; each
+    # linear waits only for its own inputs.
     e2e = None
     if not args.no_e2e:
-        host_x = [l["x"].cpu().pin_memory() for l in layers]
+        srcs = sorted({l["x_src"] for l in layers})
+        host_x = {j: layers[j]["x"].cpu().pin_memory() for j in srcs}
         host_dz = [l["dz"].cpu().pin_memory() for l in layers]
         host_dq = torch.empty(flat.numel(), dtype=torch.float32).pin_memory()
-        h2d = sum(t.numel() * t.element_size() for t in host_x + host_dz)
+        h2d = sum(t.numel() * t.element_size() for t in list(host_x.values()) + host_dz)
         d2h = host_dq.numel() * 4
         e_steps = max(2, min(args.steps, 6))
         copy_stream = torch.cuda.Stream(device)
-        dev_x = [[l["x"] for l in layers], [torch.empty_like(l["x"]) for l in layers]]
+        dev_x = [{j: layers[j]["x"] for j in srcs}, {j: torch.empty_like(layers[j]["x"]) for j in srcs}]
         dev_dz = [[l["dz"] for l in layers], [torch.empty_like(l["dz"]) for l in layers]]
+        readers = {j: [i for i, l in enumerate(layers) if l["x_src"] == j] for j in srcs}
         ev = lambda: torch.cuda.Event()  # noqa: E731
-        x_ready = [[ev() for _ in layers] for _ in range(2)]
+        x_ready = [{j: ev() for j in srcs} for _ in range(2)]
         dz_ready = [[ev() for _ in layers] for _ in range(2)]
         consumed = [[ev() for _ in layers] for _ in range(2)]
         for k in range(2):
@@ -400,23 +411,25 @@ def bench_poetx(args, cfg: pi.Config) -> dict:
 
         def e2e_step(k):
             with torch.cuda.stream(copy_stream):
-                for i, l in enumerate(layers):
-                    copy_stream.wait_event(consumed[k][i])
-                    dev_x[k][i].copy_(host_x[i], non_blocking=True)
-                    x_ready[k][i].record(copy_stream)
+                for j in srcs:
+                    for i in readers[j]:
+                        copy_stream.wait_event(consumed[k][i])
+                    dev_x[k][j].copy_(host_x[j], non_blocking=True)
+                    x_ready[k][j].record(copy_stream)
                 for i in reversed(range(len(layers))):
                     dev_dz[k][i].copy_(host_dz[i], non_blocking=True)
                     dz_ready[k][i].record(copy_stream)
 
             def ready(i, kind):
                 if kind == "x":
-                    stream.wait_event(x_ready[k][i])
+                    stream.wait_event(x_ready[k][layers[i]["x_src"]])
                 elif kind == "dz":
                     stream.wait_event(dz_ready[k][i])
                 else:
                     consumed[k][i].record(stream)
 
-            run_step(layers, flat, xs=dev_x[k], dzs=dev_dz[k], ready=ready)
+            xs = [dev_x[k][l["x_src"]] for l in layers]
+            run_step(layers, flat, xs=xs, dzs=dev_dz[k], ready=ready)
             host_dq.copy_(flat, non_blocking=True)
 
         e2e_step(0)
@@ -455,10 +468,15 @@ def bench_poetx(args, cfg: pi.Config) -> dict:
         def step_mem():
             run_step(layers, flat, mem=True)
 
+        # each variant is timed right after the plain step over the same
+        # number of steps ("base_ms_per_step"), so that the pair shares the
+        # board's power and thermal state (it drifts over a run at the cap)
+        base = lambda: run_step(layers, flat)  # noqa: E731
         variants = {}
         step_mem()
+        ms_b = timed(base, args.steps)
         ms = timed(step_mem, args.steps)
-        variants["mem"] = {"tokens_per_s": world * cfg.T / (ms / 1e3), "ms_per_step": ms,
+        variants["mem"] = {"tokens_per_s": world * cfg.T / (ms / 1e3), "ms_per_step": ms, "base_ms_per_step": ms_b,
                            "note": "backward recomputes Y; no [T][n] activation kept"}
         group = layers[0]["group"]
         opt = lambda: group.optimizer_step(flat, 1e-4, weight_decay=0.0)  # noqa: E731
@@ -466,13 +484,21 @@ def bench_poetx(args, cfg: pi.Config) -> dict:
         ms = timed(opt, args.steps)
         variants["optimizer_step"] = {"ms_per_step": ms, "params": int(group.q.numel()),
                                       "note": "AdamW on every packed triangle + batched CNP rebuild of every G"}
+        ms_b = timed(base, args.steps)
         scratch = torch.empty(max(l["m"] * l["n"] for l in layers), dtype=torch.bfloat16, device=device)
         for l in layers:
             l["L"].quantize_weight(scratch)
         run_step(layers, flat)
-        ms = timed(lambda: run_step(layers, flat), args.steps)
-        variants["xq"] = {"tokens_per_s": world * cfg.T / (ms / 1e3), "ms_per_step": ms,
+        ms = timed(base, args.steps)
+        # stage breakdown of the same step (library profiler, a few steps)
+        px.poetx_profile_begin()
+        for _ in range(3):
+            run_step(layers, flat)
+        torch.cuda.synchronize(device)
+        xq_stages = px.poetx_profile_end()
+        variants["xq"] = {"tokens_per_s": world * cfg.T / (ms / 1e3), "ms_per_step": ms, "base_ms_per_step": ms_b,
                           "weight_bytes": int(sum(l["m"] * l["n"] + 4 * l["n"] for l in layers)),
+                          "stages_ms_per_step": {k: v[0] / 3 for k, v in xq_stages.items() if v[1]},
                           "note": "int8 per-row weights, dequantized into one shared scratch before each use"}
     device_error = px.poetx_device_error()
 

@@ -40,6 +40,12 @@ class Config:
     dtype: str          # "fp32" or "bf16": storage type of x, W0, dz, G, z, dx
     sigma_q: float
     description: str
+    # x_from[i]: the linear whose input linear i reads (a decoder block's q, k,
+    # v read one normalised hidden state, gate and up another); () = each its own
+    x_from: Tuple[int, ...] = ()
+
+    def x_source(self, layer: int) -> int:
+        return self.x_from[layer] if self.x_from else layer
 
     def flops_per_step(self) -> float:
         """Algorithmic flops of one forward+backward step (no merge).
@@ -73,7 +79,8 @@ CONFIGS = {
                        ("o", 4096, 4096), ("gate", 4096, 14336), ("up", 4096, 14336),
                        ("down", 14336, 4096)),
                       256, 16384, "bf16", 0.01,
-                      "Llama-8B decoder block, 7 linears in sequence, b=256, T=16384"),
+                      "Llama-8B decoder block, 7 linears in sequence, b=256, T=16384; q/k/v read one input, "
+                      "gate/up another", x_from=(0, 0, 0, 3, 4, 4, 6)),
 }
 
 
