@@ -37,7 +37,9 @@
  *  - dtype POETX_BF16: x, z, W, G, y_save, dz, dx are bf16, accumulation is
  *    fp32 on tcgen05 tensor cores; b must be a multiple of 64.  dtype
  *    POETX_FP32: everything fp32 (FFMA; tcgen05 has no fp32 kind).
- *  - Requirements: b >= 2 divides m and n; the device is compute capability
+ *  - Requirements: b >= 2 divides m and n; m <= 51200 and n <= 102400 (bf16)
+ *    or 51200 (fp32), the widest rows the row-staging kernels hold in shared
+ *    memory; T <= 2^31 - 257 token rows; the device is compute capability
  *    10.0 (B200).
  */
 #ifndef POETX_H
@@ -53,7 +55,7 @@ extern "C" {
 typedef enum {
   POETX_OK = 0,
   POETX_E_ARG = 1,       /* null pointer, negative size, bad flag */
-  POETX_E_SHAPE = 2,     /* b does not divide m or n, b unsupported for the dtype */
+  POETX_E_SHAPE = 2,     /* b does not divide m or n, b unsupported for the dtype, m, n or T above its limit */
   POETX_E_DTYPE = 3,     /* unknown dtype */
   POETX_E_ALIGN = 4,     /* a pointer is not 16-byte aligned */
   POETX_E_WORKSPACE = 5, /* ws too small or NULL */
@@ -88,7 +90,8 @@ int32_t poetx_version(void);
  * it.  Synchronises the current device. */
 poetx_status poetx_device_error(uint32_t* code);
 
-/* Workspace sizes in bytes (host-side arithmetic only, no device access). */
+/* Workspace sizes in bytes (host-side arithmetic only, no device access);
+ * 0 for an invalid layer or T. */
 size_t poetx_cnp_workspace_bytes(int32_t nblk, int32_t b, int32_t dtype);
 size_t poetx_forward_workspace_bytes(const poetx_layer* layer, int64_t T);
 size_t poetx_backward_workspace_bytes(const poetx_layer* layer, int64_t T);

@@ -33,6 +33,13 @@ inline size_t al(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline int dtype_size(int32_t dt) { return dt == POETX_BF16 ? 2 : 4; }
 inline int elem_type(int32_t dt) { return dt == POETX_BF16 ? ET_BF16 : ET_F32; }
+// Widest rows the row-staging kernels take (one row of at most 200 KB in
+// shared memory): n for the activation permutations (rows of the layer dtype),
+// m also for the merge, whose reframing gather reads fp32 rows of length m.
+constexpr int32_t kMaxM = 51200;
+inline int32_t max_n(int32_t dt) { return dt == POETX_BF16 ? 102400 : 51200; }
+// Token rows: GEMM row counts and TMA row coordinates are 32-bit.
+constexpr int64_t kMaxT = 2147483647 - 256;
 
 struct Carver {
   uint8_t* base;
@@ -99,6 +106,7 @@ poetx_status check_layer(const poetx_layer* L) {
   if (!L) return POETX_E_ARG;
   POETX_TRY(check_dtype_b(L->dtype, L->b));
   if (L->m <= 0 || L->n <= 0 || L->m % L->b != 0 || L->n % L->b != 0) return POETX_E_SHAPE;
+  if (L->m > kMaxM || L->n > max_n(L->dtype)) return POETX_E_SHAPE;
   const void* ptrs[] = {L->W, L->permR, L->permP, L->qR, L->qP, L->GR, L->GP};
   for (const void* p : ptrs) {
     if (!p) return POETX_E_ARG;
@@ -318,7 +326,11 @@ cudaError_t permute_cols(const T* in, T* out, int64_t rows, int cols, const int3
   if (rps > 64) rps = 64;
   const size_t idx_bytes = (size_t(cols) * 2 + 127) & ~size_t(127);
   const size_t smem = idx_bytes + 2 * size_t(rps) * row_bytes;
-  if (smem > 200 * 1024) return cudaErrorInvalidValue;
+  if (smem > 200 * 1024) {
+    // rows too wide for two staged rows and the index table: one row at a time
+    return inverse ? scatter(in, cols, out, cols, rows, rows, cols, map, nullptr, st, device)
+                   : gather(in, cols, rows, out, cols, rows, cols, map, nullptr, st, device);
+  }
   cudaError_t e = allow_smem(permute_rows_kernel<T>, smem, &attr[device & 63]);
   if (e != cudaSuccess) return e;
   const int per_sm = static_cast<int>((220 * 1024) / (smem + 1024));
@@ -1036,17 +1048,17 @@ poetx_status poetx_layer_cnp_build(const poetx_layer* layer, void* ws, size_t ws
 }
 
 size_t poetx_forward_workspace_bytes(const poetx_layer* layer, int64_t T) {
-  if (check_layer(layer) != POETX_OK || T < 0) return 0;
+  if (check_layer(layer) != POETX_OK || T < 0 || T > kMaxT) return 0;
   return fwd_ws(layer, T);
 }
 
 size_t poetx_backward_workspace_bytes(const poetx_layer* layer, int64_t T) {
-  if (check_layer(layer) != POETX_OK || T < 0) return 0;
+  if (check_layer(layer) != POETX_OK || T < 0 || T > kMaxT) return 0;
   return bwd_ws(layer, T);
 }
 
 size_t poetx_backward_recompute_workspace_bytes(const poetx_layer* layer, int64_t T) {
-  if (check_layer(layer) != POETX_OK || T < 0) return 0;
+  if (check_layer(layer) != POETX_OK || T < 0 || T > kMaxT) return 0;
   return bwd_recompute_ws(layer, T);
 }
 
@@ -1118,6 +1130,7 @@ poetx_status poetx_forward(const poetx_layer* layer, int64_t T, const void* x, v
                            void* xg_save, void* ws, size_t ws_bytes, void* stream) {
   POETX_TRY(check_layer(layer));
   if (T < 0) return POETX_E_ARG;
+  if (T > kMaxT) return POETX_E_SHAPE;
   if (T == 0) return POETX_OK;
   POETX_TRY(check_ptr(x));
   POETX_TRY(check_ptr(z));
@@ -1193,6 +1206,7 @@ static poetx_status backward_impl(const poetx_layer* layer, int64_t T, const voi
                            float* dGP, int32_t accumulate, void* ws, size_t ws_bytes, void* stream) {
   POETX_TRY(check_layer(layer));
   if (T < 0) return POETX_E_ARG;
+  if (T > kMaxT) return POETX_E_SHAPE;
   const bool dg_mode = dGR != nullptr;
   const poetx_layer& L = *layer;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

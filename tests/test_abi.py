@@ -66,6 +66,12 @@ def test_workspace_sizes_are_host_arithmetic(lib):
     assert px.poetx_forward_workspace_bytes(_layer(b=48), T) == 0   # bf16 needs b % 64 == 0
     assert px.poetx_forward_workspace_bytes(_layer(m=500), T) == 0  # b must divide m
     assert px.poetx_forward_workspace_bytes(_layer(dtype=7), T) == 0
+    # row and token limits (one staged row of at most 200 KB; 32-bit row counts)
+    assert px.poetx_forward_workspace_bytes(_layer(m=51200, n=102400, b=256), T) > 0
+    assert px.poetx_forward_workspace_bytes(_layer(m=51456, b=256), T) == 0
+    assert px.poetx_forward_workspace_bytes(_layer(n=102656, b=256), T) == 0
+    assert px.poetx_forward_workspace_bytes(_layer(n=51264, b=64, dtype=px.POETX_FP32), T) == 0
+    assert px.poetx_forward_workspace_bytes(_layer(), 2 ** 31) == 0
 
 
 def test_validation_before_any_launch(lib):
@@ -79,6 +85,11 @@ def test_validation_before_any_launch(lib):
     assert lib.poetx_forward(ctypes.byref(L), 10, 4096, 4096, None, None, 4096, 1 << 30, None) == 4  # E_ALIGN
     L = _layer()
     assert lib.poetx_forward(ctypes.byref(L), -1, 4096, 4096, None, None, 4096, 1 << 30, None) == 1  # T < 0
+    assert lib.poetx_forward(ctypes.byref(L), 2 ** 31, 4096, 4096, None, None, 4096, 1 << 30, None) == 2  # T big
+    Lw = _layer(m=51456, b=256)
+    assert lib.poetx_forward(ctypes.byref(Lw), 10, 4096, 4096, None, None, 4096, 1 << 30, None) == 2  # m wide
+    assert lib.poetx_backward_dG(ctypes.byref(L), 2 ** 31, 4096, 4096, None, 4096, None, 4096, 4096, 0, 4096,
+                                 1 << 30, None) == 2                                          # T big
     assert lib.poetx_forward(ctypes.byref(L), 10, 4096, 4096, None, None, 4096, 16, None) == 5       # ws small
     assert lib.poetx_forward(ctypes.byref(L), 10, None, 4096, None, None, 4096, 1 << 30, None) == 1  # x NULL
     assert lib.poetx_backward(ctypes.byref(L), 10, 4096, 4100, None, 4096, None, 4096, 4096, 0, 4096, 1 << 30,

@@ -230,6 +230,25 @@ def test_merge_with_zero_q_is_exact_reframing(dtype):
     assert np.array_equal(bits(L.W), want.view(np.uint16 if dtype == "bf16" else np.uint32))
 
 
+@pytest.mark.parametrize("m,n", [(36864, 256), (256, 40960)], ids=["wide-m", "wide-n"])
+def test_wide_rows_take_the_one_row_permutation(m, n):
+    # bf16 rows wider than the double-buffered permutation holds with its index
+    # table (about 34K columns) go through the kernels that stage one row at a
+    # time: frame bit-exact, layer and merge against the oracle
+    inp = _inputs("up8b", m, n, 256, 72)
+    L = make_layer(inp)
+    torch.cuda.synchronize()
+    want = oracle.to_frame(inp.W0lin, inp.permR, inp.permP)
+    assert np.array_equal(bits(L.W), want.view(np.uint16))
+    z, _, dx, dqR, dqP = _run(L, inp)
+    zo, dxo, dqRo, dqPo, _, _ = _oracle_all(inp)
+    check(host64(z), zo, "bf16", "z (wide)")
+    check(host64(dx), dxo, "bf16", "dx (wide)")
+    check(host64(dqR), dqRo, "bf16", "dqR (wide)")
+    check(host64(dqP), dqPo, "bf16", "dqP (wide)")
+    _merge_check(inp)
+
+
 def test_empty_and_single_token():
     inp = _inputs("attn3b", 512, 512, 256, 1)
     L = make_layer(inp)
