@@ -23,6 +23,22 @@ from . import (POETX_BF16, POETX_FP32, make_layer, poetx_backward, poetx_backwar
 _TORCH_DTYPE = {POETX_BF16: torch.bfloat16, POETX_FP32: torch.float32}
 
 
+def _need(t, shape, dtype, device: torch.device, name: str) -> None:
+    """Host-side check of a tensor handed to the library.  The C calls take
+    raw device pointers and trust the layer's sizes, so a tensor of another
+    shape, dtype, device or stride must be refused here, before any launch."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
+    if t.device.type != device.type or (device.index is not None and t.device.index != device.index):
+        raise ValueError(f"{name}: tensor on {t.device}, the layer is on {device}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+
+
 class Saved(NamedTuple):
     """Activations the forward keeps for the backward: Y ([T][n], the P-side
     input in the Psi_P frame) and optionally Xg ([T][m], x in the Psi_R frame)."""
@@ -63,6 +79,9 @@ class PoetxLinear:
         poetx_weight_quantize(self.n, self.m, self.W, self.dtype, self.Wq, self.Wscale, stream)
         if scratch is None:
             scratch = torch.empty(self.n * self.m, dtype=self.torch_dtype, device=self.device)
+        if scratch.numel() < self.n * self.m:
+            raise ValueError(f"scratch: {scratch.numel()} elements, the layer needs {self.n * self.m}")
+        _need(scratch, (scratch.numel(),), self.torch_dtype, self.device, "scratch")
         self._wscratch = scratch
         self.W = scratch[: self.n * self.m].view(self.n, self.m)
 
@@ -91,11 +110,17 @@ class PoetxLinear:
              qP: torch.Tensor, stream=None) -> None:
         """Set the permutations and triangles, import the natural nn.Linear
         weight W0^T ([n][m]) into the frame, and build G."""
+        W0lin = W0lin.contiguous()
+        _need(W0lin, (self.n, self.m), self.torch_dtype, self.device, "W0lin")
+        for name, t, shape in (("permR", permR, self.permR.shape), ("permP", permP, self.permP.shape),
+                               ("qR", qR, self.qR.shape), ("qP", qP, self.qP.shape)):
+            if tuple(t.shape) != tuple(shape):
+                raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
         self.permR.copy_(permR)
         self.permP.copy_(permP)
         self.qR.copy_(qR)
         self.qP.copy_(qP)
-        poetx_frame_import(self.abi(), W0lin.contiguous(), stream)
+        poetx_frame_import(self.abi(), W0lin, stream)
         self.build(stream)
 
     def export_weight(self, stream=None) -> torch.Tensor:
@@ -117,14 +142,21 @@ class PoetxLinear:
         """z = x R W0 P.  With `save`, also returns what the backward needs:
         Y (the P-side input) and, with `save_xg`, Xg = x[:, permR]."""
         T = x.shape[0]
+        td = self.torch_dtype
+        _need(x, (T, self.m), td, self.device, "x")
         if z is None:
-            z = torch.empty((T, self.n), dtype=self.torch_dtype, device=self.device)
+            z = torch.empty((T, self.n), dtype=td, device=self.device)
+        _need(z, (T, self.n), td, self.device, "z")
         if save and y is None:
-            y = torch.empty((T, self.n), dtype=self.torch_dtype, device=self.device)
+            y = torch.empty((T, self.n), dtype=td, device=self.device)
+        if save:
+            _need(y, (T, self.n), td, self.device, "y")
         if save and save_xg and xg is None:
-            xg = torch.empty((T, self.m), dtype=self.torch_dtype, device=self.device)
+            xg = torch.empty((T, self.m), dtype=td, device=self.device)
         if not (save and save_xg):
             xg = None
+        if xg is not None:
+            _need(xg, (T, self.m), td, self.device, "xg")
         self._dequantize(stream)
         L = self.abi()
         nb = poetx_forward_workspace_bytes(L, T)
@@ -149,6 +181,9 @@ class PoetxLinear:
             dqR = torch.empty_like(self.qR)
         if dqP is None:
             dqP = torch.empty_like(self.qP)
+        self._check_backward(T, x, saved, dz, dx if need_dx else None)
+        _need(dqR, tuple(self.qR.shape), torch.float32, self.device, "dqR")
+        _need(dqP, tuple(self.qP.shape), torch.float32, self.device, "dqP")
         self._dequantize(stream)
         L = self.abi()
         nb = (poetx_backward_workspace_bytes if saved.y is not None else poetx_backward_recompute_workspace_bytes)(L, T)
@@ -170,6 +205,9 @@ class PoetxLinear:
         T = dz.shape[0]
         if need_dx and dx is None:
             dx = torch.empty((T, self.m), dtype=self.torch_dtype, device=self.device)
+        self._check_backward(T, x, saved, dz, dx if need_dx else None)
+        _need(dGR, (self.m // self.b, self.b, self.b), torch.float32, self.device, "dGR")
+        _need(dGP, (self.n // self.b, self.b, self.b), torch.float32, self.device, "dGP")
         self._dequantize(stream)
         L = self.abi()
         nb = (poetx_backward_workspace_bytes if saved.y is not None else poetx_backward_recompute_workspace_bytes)(L, T)
@@ -177,6 +215,20 @@ class PoetxLinear:
         poetx_backward_dG(L, T, x, saved.y, saved.xg, dz, dx if need_dx else None, dGR, dGP, int(accumulate), ws, nb,
                           stream)
         return dx if need_dx else None
+
+    def _check_backward(self, T: int, x, saved: "Saved", dz, dx) -> None:
+        td = self.torch_dtype
+        _need(dz, (T, self.n), td, self.device, "dz")
+        if x is not None:
+            _need(x, (T, self.m), td, self.device, "x")
+        elif saved.xg is None:
+            raise ValueError("x: needed unless the forward saved Xg")
+        if saved.y is not None:
+            _need(saved.y, (T, self.n), td, self.device, "saved y")
+        if saved.xg is not None:
+            _need(saved.xg, (T, self.m), td, self.device, "saved xg")
+        if dx is not None:
+            _need(dx, (T, self.m), td, self.device, "dx")
 
     def merge(self, new_permR: torch.Tensor, new_permP: torch.Tensor, stream=None) -> None:
         """W0 <- R W0 P, re-expressed in the frame of the new permutations;
@@ -187,6 +239,8 @@ class PoetxLinear:
         W_out = torch.empty_like(self.W)
         newR = new_permR.to(device=self.device, dtype=torch.int32).contiguous()
         newP = new_permP.to(device=self.device, dtype=torch.int32).contiguous()
+        _need(newR, (self.m,), torch.int32, self.device, "new_permR")
+        _need(newP, (self.n,), torch.int32, self.device, "new_permP")
         poetx_merge(L, newR, newP, W_out, ws, nb, stream)
         self.W = W_out
         self.permR.copy_(newR)
@@ -232,6 +286,7 @@ class LayerGroup:
         (same layout), then the batched CNP rebuild of every G."""
         if self.q is None:
             raise RuntimeError("flatten_params() first")
+        _need(grad, tuple(self.q.shape), torch.float32, self.q.device, "grad")
         self.steps += 1
         poetx_adamw_step(self.q.numel(), self.q, grad, self.m1, self.m2, lr, beta1, beta2, eps, weight_decay,
                          self.steps, stream)
@@ -259,7 +314,9 @@ class LayerGroup:
         if self.q is None:
             raise RuntimeError("flatten_params() first")
         L0 = self.layers[0]
-        nblk = dG.shape[0]
+        nblk = sum(L.m // L.b + L.n // L.b for L in self.layers)
+        _need(dG, (nblk, L0.b, L0.b), torch.float32, self.q.device, "dG")
+        _need(dq, tuple(self.q.shape), torch.float32, self.q.device, "dq")
         nb = poetx_cnp_workspace_bytes(nblk, L0.b, L0.dtype)
         if self._bws is None or self._bws.numel() < nb:
             self._bws = torch.empty(max(nb, 1), dtype=torch.uint8, device=L0.device)
