@@ -326,6 +326,10 @@ def bench_poetx(args, cfg: pi.Config) -> dict:
 
     rank, world, local = dist_env()
     if world > 1:
+        # NVSwitch multicast (NVLS) off unless the caller sets it: the exchange
+        # is a few tens of MB overlapped with the backward, and a rank that
+        # exits while bound to a multicast object can disturb its peers
+        os.environ.setdefault("NCCL_NVLS_ENABLE", "0")
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     device = torch.device("cuda", local)

@@ -86,8 +86,9 @@ int32_t poetx_version(void);
 
 /* Reads the sticky device error word (bit 1: a bounded wait inside a GEMM
  * timed out; bit 2: a bounded wait inside a copy kernel timed out; bit 4: a
- * permutation index was out of range) into *code (HOST pointer) and clears
- * it.  Synchronises the current device. */
+ * permutation index was out of range; bit 8, builds with -DPOETX_DEBUG only:
+ * a TMA or bulk copy broke an alignment or coordinate rule and was skipped)
+ * into *code (HOST pointer) and clears it.  Synchronises the current device. */
 poetx_status poetx_device_error(uint32_t* code);
 
 /* Workspace sizes in bytes (host-side arithmetic only, no device access);

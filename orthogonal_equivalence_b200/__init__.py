@@ -16,7 +16,8 @@ import os
 from typing import Optional
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libpoetx.so")
+# POETX_DEBUG=1 selects the build with device-side copy checks (build.py debug=True)
+LIB_PATH = os.path.join(_HERE, "libpoetx_debug.so" if os.environ.get("POETX_DEBUG") == "1" else "libpoetx.so")
 
 POETX_FP32 = 0
 POETX_BF16 = 1
@@ -84,7 +85,8 @@ def lib() -> ctypes.CDLL:
     global _lib
     if _lib is None:
         if not os.path.exists(LIB_PATH):
-            raise RuntimeError(f"libpoetx.so not built ({LIB_PATH}); run orthogonal_equivalence_b200/build.py")
+            raise RuntimeError(f"{os.path.basename(LIB_PATH)} not built ({LIB_PATH}); run "
+                               "orthogonal_equivalence_b200/build.py")
         L = ctypes.CDLL(LIB_PATH)
         for name, (res, args) in SIGNATURES.items():
             fn = getattr(L, name)

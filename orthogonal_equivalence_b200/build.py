@@ -1,7 +1,11 @@
 """Build libpoetx.so (the POET-X layer's C ABI and its sm_100a kernels) in
-place, next to this file, with nvcc."""
+place, next to this file, with nvcc; `debug=True` builds libpoetx_debug.so,
+the same library compiled with -DPOETX_DEBUG (every TMA and bulk copy checked
+before it is issued; see csrc/ptx.cuh), loaded instead when the environment
+sets POETX_DEBUG=1."""
 from __future__ import annotations
 
+import glob
 import os
 import subprocess
 import sys
@@ -10,8 +14,13 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libpoetx.so")
+LIB_DEBUG = os.path.join(HERE, "libpoetx_debug.so")
 SOURCES = ["poetx.cu"]
-DEPS = ["poetx.cu", "ptx.cuh", "gemm.cuh", "gemm_host.cuh", "perm.cuh", "cnp.cuh", "quant.cuh", "adamw.cuh", "gemm2sm.cuh"]
+
+
+def deps():
+    return (sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh"))) +
+            [os.path.join(ROOT, "include", "poetx.h")])
 
 
 def nvcc() -> str:
@@ -21,33 +30,34 @@ def nvcc() -> str:
     return "nvcc"
 
 
-def needs_build() -> bool:
-    if not os.path.exists(LIB):
+def needs_build(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
-    deps = [os.path.join(CSRC, d) for d in DEPS] + [os.path.join(ROOT, "include", "poetx.h")]
-    return any(os.path.getmtime(d) > t for d in deps if os.path.exists(d))
+    t = os.path.getmtime(lib)
+    return any(os.path.getmtime(d) > t for d in deps() if os.path.exists(d))
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not needs_build():
-        return LIB
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    lib = LIB_DEBUG if debug else LIB
+    if not force and not needs_build(lib):
+        return lib
     cmd = [nvcc(), "-std=c++17", "-O3", "-lineinfo", "-gencode", "arch=compute_100a,code=sm_100a",
            "-shared", "-Xcompiler", "-fPIC", "-I", os.path.join(ROOT, "include"), "-I", CSRC,
-           "-o", LIB + ".tmp"] + [os.path.join(CSRC, s) for s in SOURCES] + ["-lcudart"]
+           "-o", lib + ".tmp"] + [os.path.join(CSRC, s) for s in SOURCES] + ["-lcudart"]
+    if debug:
+        cmd.insert(1, "-DPOETX_DEBUG")
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd), flush=True)
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         sys.stderr.write(r.stdout + r.stderr)
-        raise RuntimeError("nvcc failed building libpoetx.so")
+        raise RuntimeError(f"nvcc failed building {os.path.basename(lib)}")
     if verbose:
         sys.stderr.write(r.stderr)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(lib + ".tmp", lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose="-v" in sys.argv)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, debug="--debug" in sys.argv))

@@ -171,6 +171,7 @@ __device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
 }
 
 __device__ __forceinline__ void bulk_store(void* dst, uint32_t src, uint32_t bytes) {
+  if (!copy_ok(((src | bytes) & 15u) == 0 && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0)) return;
   asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src), "r"(bytes)
                : "memory");
 }

@@ -62,6 +62,7 @@ __device__ __forceinline__ void remote_arrive(uint32_t cluster_addr) {
 // leader CTA's barrier (cluster address); no multicast.
 __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void* tmap, uint32_t bar_cluster, int32_t c0,
                                                  int32_t c1) {
+  if (!copy_ok((c0 & 3) == 0 && (dst & 127u) == 0)) return;
   asm volatile(
       "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),

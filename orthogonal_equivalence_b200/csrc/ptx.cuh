@@ -21,9 +21,29 @@ enum DeviceError : unsigned int {
   DERR_GEMM_WAIT = 1u,      // an mbarrier wait in the tensor-core GEMM timed out
   DERR_PERM_WAIT = 2u,      // a bulk-copy wait in a permutation kernel timed out
   DERR_BAD_INDEX = 4u,      // a permutation index was out of range (access skipped)
+  DERR_DEBUG_CHECK = 8u,    // (POETX_DEBUG builds) a copy broke an alignment or coordinate rule (copy skipped)
 };
 
 __device__ __forceinline__ void record_error(unsigned int code) { atomicOr(&g_device_error, code); }
+
+// Debug builds (-DPOETX_DEBUG) check every TMA and bulk copy before issuing
+// it: the innermost coordinate a multiple of 16 bytes (4 elements is the
+// weakest such rule over the 2- and 4-byte types used here), no store at a
+// negative coordinate, 128-byte aligned shared-memory tiles, 16-byte aligned
+// addresses and sizes for untiled bulk copies.  A copy that fails is skipped
+// and DERR_DEBUG_CHECK recorded (its consumer's bounded wait then times out).
+// In release builds the checks compile away.
+__device__ __forceinline__ bool copy_ok(bool cond) {
+#ifdef POETX_DEBUG
+  if (!cond) {
+    record_error(DERR_DEBUG_CHECK);
+    return false;
+  }
+#else
+  (void)cond;
+#endif
+  return true;
+}
 
 __device__ __forceinline__ uint64_t global_ns() {
   uint64_t t;
@@ -92,6 +112,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigne
 // ---------------------------------------------------------------- TMA (no multicast)
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, uint32_t bar, int32_t c0,
                                             int32_t c1) {
+  if (!copy_ok((c0 & 3) == 0 && (dst & 127u) == 0)) return;
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
@@ -101,6 +122,7 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, uint
 
 // TMA tensor store shared -> global (no multicast), tracked by bulk groups.
 __device__ __forceinline__ void tma_store_2d(const void* tmap, uint32_t src, int32_t c0, int32_t c1) {
+  if (!copy_ok((c0 & 3) == 0 && c0 >= 0 && c1 >= 0 && (src & 127u) == 0)) return;
   asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(tmap),
                "r"(src), "r"(c0), "r"(c1)
                : "memory");
@@ -121,6 +143,7 @@ __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
 
 // Plain bulk copy global -> shared (16-byte aligned, size multiple of 16).
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  if (!copy_ok(((dst | bytes) & 15u) == 0 && (reinterpret_cast<uintptr_t>(src) & 15u) == 0)) return;
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
       "l"(src), "r"(bytes), "r"(bar)

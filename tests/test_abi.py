@@ -122,3 +122,11 @@ def test_no_device_call_fails_cleanly(lib):
     T = 10
     ws = px.poetx_forward_workspace_bytes(L, T)
     assert lib.poetx_forward(ctypes.byref(L), T, 4096, 4096, 4096, None, 4096, ws, None) == 7
+
+
+def test_debug_build_exports_the_same_symbols(lib):
+    # -DPOETX_DEBUG (device-side copy checks) changes no symbol of the ABI
+    path = pbuild.build(debug=True)
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (poetx_\w+)", out))
+    assert set(header_functions()) <= exported
