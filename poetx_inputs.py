@@ -22,7 +22,7 @@ k-th merge adds 100*k.
 from __future__ import annotations
 
 import dataclasses
-from typing import List, Tuple
+from typing import Tuple
 
 import numpy as np
 
@@ -182,7 +182,3 @@ def random_token_rows(seed: int, T: int, count: int) -> np.ndarray:
     rows = g.choice(T, size=min(count, T), replace=False)
     rows[-1] = T - 1
     return np.unique(rows).astype(np.int64)
-
-
-def layers_of(cfg: Config) -> List[Tuple[str, int, int]]:
-    return list(cfg.layers)
