@@ -14,7 +14,15 @@ next linear's backward; the CNP backward is linear in dG, so this gives the
 summed dq.  Each rank processes its own 16384 tokens (weak
 scaling).  Inputs are synthetic (seeded normal activations / gradients,
 N(0, 0.02^2) weights, N(0, 0.01^2) triangles, seeded permutations), drawn on
-the device; every tensor of the working set is larger than L2.
+the device; q, k, v read one input and gate, up another, as in the decoder
+block; every tensor of the working set is larger than L2.
+
+The JSON line also carries: the end-to-end rate through the Python API with
+every step's inputs copied from pinned host memory and the dq read back
+("e2e"); the stage breakdown from the library's profiler; the dominant
+kernel's roofline; nvidia-smi clocks, reasons and power stamped inside the
+timed region; and the mem / POET-XQ variants and the optimizer step, each
+variant timed right after a fresh timing of the plain step.
 
 --impl reference times the float64 CPU oracle (oracle/) on the host cores on
 a bounded token sample of the same workload.
