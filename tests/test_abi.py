@@ -5,6 +5,7 @@ import ctypes
 import os
 import re
 import subprocess
+import sys
 
 import pytest
 
@@ -130,3 +131,13 @@ def test_debug_build_exports_the_same_symbols(lib):
     out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True).stdout
     exported = set(re.findall(r"\bT (poetx_\w+)", out))
     assert set(header_functions()) <= exported
+
+
+def test_debug_environment_selects_the_debug_library():
+    # POETX_DEBUG=1 makes the package load libpoetx_debug.so; otherwise libpoetx.so
+    code = "import orthogonal_equivalence_b200 as px; print(os.path.basename(px.LIB_PATH))"
+    for flag, want in (("1", "libpoetx_debug.so"), ("0", "libpoetx.so")):
+        env = dict(os.environ, POETX_DEBUG=flag)
+        out = subprocess.run([sys.executable, "-c", "import os; " + code], cwd=ROOT, env=env, capture_output=True,
+                             text=True).stdout.strip()
+        assert out == want, (flag, out)
