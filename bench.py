@@ -7,7 +7,10 @@ Llama-8B decoder block's seven linears (q, k, v, o, gate, up, down; b = 256,
 One step = the G_R, G_P blocks of every linear built from the packed triangles
 (one batched CNP build), the forwards (saving Y and the gathered input), the
 backwards in reverse order (dx and the token sums dG of both sides), then one
-batched CNP backward from the dG of all linears to their packed dq.  With N > 1
+batched CNP backward from the dG of all linears to their packed dq.  The
+headline step is input-centric (the write-up's section 1): every block product
+acts on token rows and no transformed weight is formed; the weight-fold and
+weight-centric evaluations are reported as labelled variants.  With N > 1
 ranks each linear's dG is summed across ranks (NCCL all-reduce, the
 data-parallel exchange) as soon as its backward is done, overlapped with the
 next linear's backward; the CNP backward is linear in dG, so this gives the
@@ -21,8 +24,11 @@ The JSON line also carries: the end-to-end rate through the Python API with
 every step's inputs copied from pinned host memory and the dq read back
 ("e2e"); the stage breakdown from the library's profiler; the dominant
 kernel's roofline; nvidia-smi clocks, reasons and power stamped inside the
-timed region; and the mem / POET-XQ variants and the optimizer step, each
-variant timed right after a fresh timing of the plain step.
+timed region; the folded / mem / POET-XQ variants and the optimizer step, each
+variant timed right after a fresh timing of the plain step; the merge of all
+seven linears; and ("configs") the single-layer workloads attn3b, up8b and
+down13b (step rate, W0 roofline, CNP build and backward microbenchmark, the
+down13b merge) and the 8B block's batched CNP microbenchmark.
 
 --impl reference times the float64 CPU oracle (oracle/) on the host cores on
 a bounded token sample of the same workload.
@@ -53,6 +59,7 @@ WORKLOAD = "block8b"
 # is captured again.
 W0_GEMM_TRAFFIC_BYTES = 1109613056 + 456707584
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+NOMINAL_BF16_TFLOPS = 2250.0   # B200 dense bf16 tensor-core peak (datasheet, no sparsity)
 
 
 def measured_peaks():
@@ -230,7 +237,7 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- POET-X arm
-def build_block(cfg: pi.Config, device, rank: int):
+def build_block(cfg: pi.Config, device, rank: int, fold: int = 0):
     import torch
     import orthogonal_equivalence_b200 as px
     layers = []
@@ -248,7 +255,7 @@ def build_block(cfg: pi.Config, device, rank: int):
         qR = torch.randn((m // cfg.b, tri), generator=g, device=device) * cfg.sigma_q
         g.manual_seed(pi.seed_of(cfg, li, "qP"))
         qP = torch.randn((n // cfg.b, tri), generator=g, device=device) * cfg.sigma_q
-        L = px.PoetxLinear(m, n, cfg.b, px.POETX_BF16, device=device)
+        L = px.PoetxLinear(m, n, cfg.b, px.POETX_BF16, device=device, fold=fold)
         L.load(W0lin, permR, permP, qR, qP)
         del W0lin
         # per-rank data (each data-parallel rank sees its own tokens); linears
@@ -322,6 +329,143 @@ def run_step(layers, flat, mem: bool = False, xs=None, dzs=None, ready=None) -> 
         pending.append(allreduce_start(l["dG_all"]))
     allreduce_finish(pending)
     group.cnp_backward(layers[0]["dG"], flat)
+
+
+def time_per_call(fn, k: int, device, stream) -> float:
+    """Mean device ms of fn() over k calls: CUDA events on the launching
+    stream between barriers + synchronizes, max over ranks."""
+    import torch
+    barrier(device)
+    a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(k):
+        fn()
+    b_.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    return reduce_max(a.elapsed_time(b_), device) / k
+
+
+def dominant_w0(cfg: pi.Config, records):
+    """The dominant kernel: the forward W0 GEMM (Y = U W~, M = T, N = n,
+    K = m) of the linears with the largest m x n and that exact shape.
+    Returns ((m, n), those linears, their per-launch ms from the profiler's
+    records of whole input-centric steps, whose W0 launches come forward in
+    layer order, then backward in reverse order)."""
+    L = len(cfg.layers)
+    big = max(m * n for _, m, n in cfg.layers)
+    shape = next((m, n) for _, m, n in cfg.layers if m * n == big)
+    dom_layers = [i for i, (_, m, n) in enumerate(cfg.layers) if (m, n) == shape]
+    w0_rec = [ms for st, ms in records if st == "w0_gemm"]
+    dom_ms = [ms for k, ms in enumerate(w0_rec) if (k % (2 * L)) < L and (k % (2 * L)) in dom_layers]
+    return shape, dom_layers, dom_ms
+
+
+def time_merges(cfg: pi.Config, plist, device, stream, k: int = 3) -> dict:
+    """One merge (W0 <- R W0 P into a scratch weight, q = 0, G = I) of every
+    layer in `plist`, timed over k repetitions (the merge's arithmetic does
+    not depend on the values, so the repetitions that start from q = 0 cost
+    the same).  Algorithmic work per layer: 4 n m b flops (the two block
+    products) and 4 n m bytes (the bf16 weight read and written)."""
+    import torch
+    import orthogonal_equivalence_b200 as px
+    nb = max(px.poetx_merge_workspace_bytes(L.abi()) for L in plist)
+    ws = torch.empty(nb, dtype=torch.uint8, device=device)
+    W_out = torch.empty(max(L.m * L.n for L in plist), dtype=torch.bfloat16, device=device)
+    perms = []
+    for i, L in enumerate(plist):
+        newR, newP = pi.merge_perms(cfg, i, 1, L.m, L.n)
+        perms.append((torch.from_numpy(newR).to(device), torch.from_numpy(newP).to(device)))
+
+    def merge_all():
+        for L, (newR, newP) in zip(plist, perms):
+            px.poetx_merge(L.abi(), newR, newP, W_out, ws, nb)
+
+    merge_all()
+    ms = time_per_call(merge_all, k, device, stream)
+    flops = sum(4.0 * L.n * L.m * L.b for L in plist)
+    nbytes = sum(4.0 * L.n * L.m for L in plist)
+    return {"layers": [f"{L.m}x{L.n}" for L in plist], "ms": ms, "tflops": flops / (ms / 1e3) / 1e12,
+            "algorithmic_gbs": nbytes / (ms / 1e3) / 1e9,
+            "note": "one merge of every listed linear: W0 <- R W0 P re-framed into new permutations, q = 0, G = I"}
+
+
+def cnp_microbench(cfg: pi.Config, device, stream, k: int = 20) -> dict:
+    """The Cayley-Neumann build of G_R, G_P of every linear of `cfg` (one
+    batch) and its backward from dG to the packed dq (one batch), timed
+    separately over k calls each.  Algorithmic flops per block: 4 b^3 for the
+    build (S = Q Q, then (2Q + S) S), 8 b^3 for the backward."""
+    import torch
+    import orthogonal_equivalence_b200 as px
+    b = cfg.b
+    Ls = []
+    for li, (_, m, n) in enumerate(cfg.layers):
+        L = px.PoetxLinear(m, n, b, px.POETX_BF16, device=device)
+        g = torch.Generator(device=device)
+        g.manual_seed(pi.seed_of(cfg, li, "qR"))
+        L.qR.copy_(torch.randn(L.qR.shape, generator=g, device=device) * cfg.sigma_q)
+        g.manual_seed(pi.seed_of(cfg, li, "qP"))
+        L.qP.copy_(torch.randn(L.qP.shape, generator=g, device=device) * cfg.sigma_q)
+        Ls.append(L)
+    group = px.LayerGroup(Ls)
+    q = group.flatten_params()
+    dG = group.dG_buffer()
+    g = torch.Generator(device=device)
+    g.manual_seed(pi.seed_of(cfg, 0, "dz"))
+    dG.copy_(torch.randn(dG.shape, generator=g, device=device))
+    dq = torch.empty_like(q)
+    nblk = dG.shape[0]
+    group.build()
+    group.cnp_backward(dG, dq)
+    build_ms = time_per_call(group.build, k, device, stream)
+    bwd_ms = time_per_call(lambda: group.cnp_backward(dG, dq), k, device, stream)
+    return {"blocks": int(nblk), "b": b, "build_us": build_ms * 1e3, "backward_us": bwd_ms * 1e3,
+            "build_tflops": 4.0 * b ** 3 * nblk / (build_ms / 1e3) / 1e12,
+            "backward_tflops": 8.0 * b ** 3 * nblk / (bwd_ms / 1e3) / 1e12,
+            "path": "fused CTA-pair kernel (bf16 operands, fp32 accumulate)" if b == 256 else
+                    "batched tcgen05 GEMM chain (tf32 operands, fp32 accumulate)",
+            "note": "q ~ N(0, sigma^2) of the workload, dG ~ N(0, 1); k calls of each, CUDA events"}
+
+
+def measure_layer_config(name: str, args, device, stream, peaks) -> dict:
+    """One single-layer workload (input-centric): the step of run_step on its
+    own layer, timed like the headline, plus its W0 GEMM roofline, the CNP
+    microbench of its blocks and (down13b) its merge."""
+    import torch
+    import orthogonal_equivalence_b200 as px
+    cfg = pi.CONFIGS[name]
+    layers, flat = build_block(cfg, device, 0)
+    for _ in range(3):
+        run_step(layers, flat)
+    k = max(3, min(args.steps, 10))
+    ms = time_per_call(lambda: run_step(layers, flat), k, device, stream)
+    px.poetx_profile_begin()
+    for _ in range(2):
+        run_step(layers, flat)
+    torch.cuda.synchronize(device)
+    stages = px.poetx_profile_end()
+    records = px.poetx_profile_records()
+    shape, _, dom_ms = dominant_w0(cfg, records)
+    dom_flops = 2.0 * cfg.T * shape[0] * shape[1]
+    w0 = dom_flops / (statistics.mean(dom_ms) / 1e3) / 1e12 if dom_ms else None
+    tflops = cfg.flops_per_step() / (ms / 1e3) / 1e12
+    burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    out = {"workload": cfg.description, "tokens_per_s": cfg.T / (ms / 1e3), "ms_per_step": ms, "steps": k,
+           "tflops": tflops, "pct_bf16_peak_nominal": 100.0 * tflops / NOMINAL_BF16_TFLOPS,
+           "stages_ms_per_step": {s_: v[0] / 2 for s_, v in stages.items() if v[1]},
+           "w0_forward": {"M": cfg.T, "N": shape[1], "K": shape[0], "tflops": w0,
+                          "frac_of_measured_burst": (w0 / burst) if w0 else None,
+                          "frac_of_nominal": (w0 / NOMINAL_BF16_TFLOPS) if w0 else None}}
+    plist = [l["L"] for l in layers]
+    for l in layers:
+        del l["L"]
+    del layers, flat
+    out["cnp"] = cnp_microbench(cfg, device, stream)
+    if name == "down13b":
+        out["merge"] = time_merges(cfg, plist, device, stream)
+    del plist
+    torch.cuda.empty_cache()
+    return out
 
 
 def bench_poetx(args, cfg: pi.Config) -> dict:
@@ -457,37 +601,52 @@ def bench_poetx(args, cfg: pi.Config) -> dict:
                "d2h_bytes_per_step": d2h, "steps": e_steps,
                "h2d_gbs": h2d * e_steps / (e_ms / 1e3) / 1e9}
     # Variants of the same step (see the POET-X write-up's three variants and
-    # its optimizer): "mem" keeps nothing between forward and backward but x
-    # (the backward recomputes Y); "xq" keeps the frozen weights as int8 codes
-    # and dequantizes each one into a shared scratch before every use; the
-    # optimizer step is AdamW on all packed triangles plus the batched CNP
-    # rebuild.
+    # its optimizer), each timed right after the plain step over the same
+    # number of steps ("base_ms_per_step"), so that the pair shares the
+    # board's power and thermal state (it drifts over a run at the cap):
+    #   folded     - both per-step weight folds (POETX_FOLD_R | POETX_FOLD_P):
+    #                G_R applied to the weight rows in the forward, G_P in the
+    #                backward (transient weight-sized copies, not input-centric)
+    #   mem        - nothing kept between forward and backward but x; the
+    #                backward recomputes Y (input-centric throughout)
+    #   mem_folded - mem with every fold, so the forward that saves nothing is
+    #                the weight-centric single GEMM
+    #   optimizer_step - AdamW on all packed triangles + batched CNP rebuild
+    #   xq         - weights kept as int8 codes, dequantized before each use
     variants = None
+    merge_block = None
     if not args.no_variants:
         def timed(fn, k):
-            barrier(device)
-            a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            for _ in range(k):
-                fn()
-            b_.record(stream)
-            torch.cuda.synchronize(device)
-            barrier(device)
-            return reduce_max(a.elapsed_time(b_), device) / k
+            return time_per_call(fn, k, device, stream)
 
-        def step_mem():
-            run_step(layers, flat, mem=True)
+        def set_fold(f):
+            for l in layers:
+                l["L"].fold = f
 
-        # each variant is timed right after the plain step over the same
-        # number of steps ("base_ms_per_step"), so that the pair shares the
-        # board's power and thermal state (it drifts over a run at the cap)
         base = lambda: run_step(layers, flat)  # noqa: E731
+        step_mem = lambda: run_step(layers, flat, mem=True)  # noqa: E731
         variants = {}
-        step_mem()
-        ms_b = timed(base, args.steps)
-        ms = timed(step_mem, args.steps)
-        variants["mem"] = {"tokens_per_s": world * cfg.T / (ms / 1e3), "ms_per_step": ms, "base_ms_per_step": ms_b,
-                           "note": "backward recomputes Y; no [T][n] activation kept"}
+        transient = int(max(2 * l["m"] * l["n"] for l in layers))
+        for vname, fold, fn, note in (
+                ("folded", px.POETX_FOLD_ALL, base,
+                 "G_R folded into the weight rows in the forward (T > n), G_P in the backward (T > m): "
+                 "weight-sized transient copies in the existing workspace; not input-centric"),
+                ("mem", 0, step_mem, "backward recomputes Y; no [T][n] activation kept; input-centric"),
+                ("mem_folded", px.POETX_FOLD_ALL, step_mem,
+                 "mem with every fold: the forward that saves nothing is one GEMM on the whole transformed "
+                 "weight (weight-centric)")):
+            set_fold(fold)
+            fn()
+            set_fold(0)
+            ms_b = timed(base, args.steps)
+            set_fold(fold)
+            ms = timed(fn, args.steps)
+            set_fold(0)
+            variants[vname] = {"tokens_per_s": world * cfg.T / (ms / 1e3), "ms_per_step": ms,
+                               "base_ms_per_step": ms_b, "fold": fold, "note": note}
+            if fold:
+                variants[vname]["transient_weight_bytes"] = transient
+                variants[vname]["extra_workspace_bytes"] = 0
         group = layers[0]["group"]
         opt = lambda: group.optimizer_step(flat, 1e-4, weight_decay=0.0)  # noqa: E731
         opt()
@@ -496,6 +655,7 @@ def bench_poetx(args, cfg: pi.Config) -> dict:
                                       "note": "AdamW on every packed triangle + batched CNP rebuild of every G"}
         ms_b = timed(base, args.steps)
         scratch = torch.empty(max(l["m"] * l["n"] for l in layers), dtype=torch.bfloat16, device=device)
+        saved_W = [l["L"].W for l in layers]
         for l in layers:
             l["L"].quantize_weight(scratch)
         run_step(layers, flat)
@@ -510,6 +670,12 @@ def bench_poetx(args, cfg: pi.Config) -> dict:
                           "weight_bytes": int(sum(l["m"] * l["n"] + 4 * l["n"] for l in layers)),
                           "stages_ms_per_step": {k: v[0] / 3 for k, v in xq_stages.items() if v[1]},
                           "note": "int8 per-row weights, dequantized into one shared scratch before each use"}
+        for l, W in zip(layers, saved_W):
+            l["L"].Wq = None
+            l["L"].W = W
+        del scratch
+        # the merge of all linears of the block (it resets q and G, so it runs last)
+        merge_block = time_merges(cfg, [l["L"] for l in layers], device, stream)
     device_error = px.poetx_device_error()
 
     peaks, peak_src = measured_peaks()
@@ -518,19 +684,12 @@ def bench_poetx(args, cfg: pi.Config) -> dict:
     w0_ms, w0_launches = stages["w0_gemm"]
     w0_flops = cfg.gemm_flops_per_step() * args.steps  # 2Tmn forward + 2Tmn backward per linear
     peak_sus = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
-    # Dominant kernel: the forward W0 GEMM (Y = U W~, M = T, N = n, K = m) of
-    # the linears with the largest m x n and that exact shape (gate and up in
-    # the 8B block).  W0 launches per step: forward in layer order, then
-    # backward in reverse order.
-    L = len(cfg.layers)
-    big = max(m * n for _, m, n in cfg.layers)
-    shape = next((m, n) for _, m, n in cfg.layers if m * n == big)
-    dom_layers = [i for i, (_, m, n) in enumerate(cfg.layers) if (m, n) == shape]
-    w0_rec = [ms for st, ms in records if st == "w0_gemm"]
-    dom_ms = [ms for k, ms in enumerate(w0_rec) if (k % (2 * L)) < L and (k % (2 * L)) in dom_layers]
+    peak_burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    shape, dom_layers, dom_ms = dominant_w0(cfg, records)
     dom_flops = 2.0 * cfg.T * shape[0] * shape[1]
     achieved = dom_flops / (statistics.mean(dom_ms) / 1e3) / 1e12 if dom_ms else None
     total_launches = int(sum(c for _, c in stages.values()))
+    tflops = flops_step / (ms_step / 1e3) / 1e12
     res = {
         "metric": METRIC,
         "value": world * cfg.T * args.steps / (ms_total / 1e3),
@@ -545,8 +704,12 @@ def bench_poetx(args, cfg: pi.Config) -> dict:
         "dtype": "bf16",
         "data": "synthetic (seeded normal activations and gradients; random-init N(0,0.02^2) weights)",
         "config": config_block(cfg, world),
-        "tflops_per_gpu": flops_step / (ms_step / 1e3) / 1e12,
-        "pct_bf16_peak": 100.0 * flops_step / (ms_step / 1e3) / 1e12 / peak_sus,
+        "evaluation": "input-centric (every block product on token rows; no transformed weight formed)",
+        "tflops_per_gpu": tflops,
+        "pct_bf16_peak": 100.0 * tflops / NOMINAL_BF16_TFLOPS,
+        "pct_bf16_peak_of": f"nominal B200 dense bf16 peak, {NOMINAL_BF16_TFLOPS:.0f} TFLOP/s",
+        "pct_bf16_peak_measured": {"burst": 100.0 * tflops / peak_burst, "sustained": 100.0 * tflops / peak_sus,
+                                   "source": f"{peak_src} bf16_tflops / bf16_tflops_sustained (cuBLAS GEMM)"},
         "roofline": {"kernel": f"w0_gemm forward, M={cfg.T} N={shape[1]} K={shape[0]} "
                                f"(layers {[cfg.layers[i][0] for i in dom_layers]})",
                      "bound": "tensor", "achieved": achieved,
@@ -554,11 +717,15 @@ def bench_poetx(args, cfg: pi.Config) -> dict:
                      "frac": (achieved / peak_sus) if achieved else None,
                      "traffic": W0_GEMM_TRAFFIC_BYTES if (cfg.name, cfg.T) == ("block8b", 16384) else None,
                      "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)",
+                     "frac_of_burst": (achieved / peak_burst) if achieved else None,
+                     "frac_of_nominal": (achieved / NOMINAL_BF16_TFLOPS) if achieved else None,
                      "launches": len(dom_ms),
                      "algorithmic_flops_per_launch": dom_flops,
                      "algorithmic_bytes_per_launch": 2.0 * (cfg.T * shape[0] + shape[0] * shape[1] + cfg.T * shape[1]),
                      "note": "achieved = 2*T*m*n per launch / mean CUDA-event launch time over the timed region; "
-                             "traffic = DRAM bytes per launch of the same kernel and shape from an ncu capture"},
+                             "traffic = DRAM bytes per launch of the same kernel and shape from an ncu capture; "
+                             "frac divides by the measured sustained cuBLAS peak, frac_of_burst by the measured "
+                             "burst peak, frac_of_nominal by the 2250 TFLOP/s datasheet figure"},
         "w0_stage": {"tflops": w0_flops / (w0_ms / 1e3) / 1e12 if w0_ms > 0 else None, "launches": w0_launches,
                      "note": "all forward and backward W0 GEMM launches of the step"},
         "stages_ms_per_step": {k: v[0] / args.steps for k, v in stages.items()},
@@ -567,12 +734,21 @@ def bench_poetx(args, cfg: pi.Config) -> dict:
         "clocks": clocks,
         "e2e": e2e,
         "variants": variants,
+        "merge": merge_block,
         "device_error": device_error,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(cfg, args.cpu_tokens)
+        res["cpu_baseline_1core"] = cpu_baseline(cfg, args.cpu_tokens_1core, threads=1)
     for l in layers:
         del l["L"]
+    del layers, flat
+    if not args.no_configs and world == 1:
+        torch.cuda.empty_cache()
+        res["configs"] = {name: measure_layer_config(name, args, device, stream, peaks)
+                          for name in ("attn3b", "up8b", "down13b")}
+        res["configs"]["block8b"] = {"cnp": cnp_microbench(cfg, device, stream)}
+        res["device_error"] = res["device_error"] | px.poetx_device_error()
     if world > 1:
         dist.barrier(device_ids=[local])
         dist.destroy_process_group()
@@ -605,12 +781,23 @@ def oracle_inputs(cfg: pi.Config, tokens: int):
     return [pi.layer_inputs(cfg, li, T=tokens) for li in range(len(cfg.layers))]
 
 
-def cpu_baseline(cfg: pi.Config, tokens: int) -> dict:
+def cpu_baseline(cfg: pi.Config, tokens: int, threads: int | None = None) -> dict:
+    """The oracle as it stands on the host cores (all BLAS threads, or
+    `threads`), one step on a `tokens`-row sample of the workload."""
     inputs = oracle_inputs(cfg, tokens)
-    t0 = time.perf_counter()
-    oracle_step(cfg, inputs)
-    dt = time.perf_counter() - t0
-    return {"value": tokens / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+    if threads is not None:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(threads):
+            t0 = time.perf_counter()
+            oracle_step(cfg, inputs)
+            dt = time.perf_counter() - t0
+        cores = threads
+    else:
+        t0 = time.perf_counter()
+        oracle_step(cfg, inputs)
+        dt = time.perf_counter() - t0
+        cores = blas_threads()
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
             "sample": f"{tokens} of {cfg.T} tokens through all {len(cfg.layers)} linears (forward, backward, "
                       f"CNP build and backward, float64), one step, {dt:.1f} s"}
 
@@ -650,8 +837,12 @@ def main(argv=None):
                     help="override the workload's tokens per GPU (smaller cases for profiler captures)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-variants", action="store_true", help="skip the mem / xq / optimizer-step timings")
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip the folded / mem / xq / optimizer-step timings and the merge")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the single-layer workloads (attn3b, up8b, down13b) and the CNP microbenchmarks")
     ap.add_argument("--cpu-tokens", type=int, default=512, help="token sample of the CPU-baseline leg")
+    ap.add_argument("--cpu-tokens-1core", type=int, default=64, help="token sample of the one-core CPU baseline")
     ap.add_argument("--ref-tokens", type=int, default=64, help="token sample per step of --impl reference")
     args = ap.parse_args(argv)
     if args.warmup < 3:

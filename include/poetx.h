@@ -65,6 +65,26 @@ typedef enum {
 
 typedef enum { POETX_FP32 = 0, POETX_BF16 = 1 } poetx_dtype;
 
+/* Evaluation order of a bf16 layer (poetx_layer.fold).  0, the default, is
+ * the write-up's input-centric form (section 1): every block product acts on
+ * token rows and no transformed weight is ever formed.  The bits below let
+ * the library apply a block product to the n x m weight instead when that
+ * moves fewer bytes; each forms a weight-sized TRANSIENT copy in the caller's
+ * workspace (never kept between calls) and gives the same product rounded at
+ * a different point.  fp32 layers ignore them.
+ *   POETX_FOLD_R: forward with T > n: W_R = W Diag(G_R)^T, Y = Xg W_R^T.
+ *   POETX_FOLD_P: backward with T > m: W_P = Diag(G_P)^T W, dU = dV W_P.
+ *   POETX_FOLD_WEIGHT_CENTRIC: a forward that saves nothing (y_save ==
+ *     xg_save == NULL) with T > 6nm/(2m+4n) forms the whole transformed
+ *     weight Psi_P^T Diag(G_P)^T W Diag(G_R)^T Psi_R and runs one GEMM (the
+ *     write-up's weight-centric form). */
+enum {
+  POETX_FOLD_R = 1,
+  POETX_FOLD_P = 2,
+  POETX_FOLD_WEIGHT_CENTRIC = 4,
+  POETX_FOLD_ALL = 7
+};
+
 /* One layer.  All pointers are device pointers owned by the caller. */
 typedef struct {
   int32_t m, n, b;      /* W0 is m x n; blocks of b x b */
@@ -76,6 +96,7 @@ typedef struct {
   float* qP;            /* [n/b][b(b-1)/2] packed triangles of Q_P (fp32) */
   void* GR;             /* [m/b][b][b] G_R blocks in dtype, written by poetx_cnp_build */
   void* GP;             /* [n/b][b][b] G_P blocks in dtype */
+  int32_t fold;         /* POETX_FOLD_* bits; 0 = input-centric (other bits: POETX_E_ARG) */
 } poetx_layer;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -129,9 +150,12 @@ poetx_status poetx_layer_cnp_build(const poetx_layer* layer, void* ws, size_t ws
  * start-up).  The paper has no counterpart: this is a deployment variant of
  * poetx_cnp_build with the same arguments (minus ws) and the same result.
  * Scratch is a 24 MiB device array inside the library, held by every GPU
- * that loads it until the process exits; it fits Q, S and H of up to
- * nblk*b*b ~= 2.09e6 fp32 elements (b = 256: nblk <= 31; b = 512: nblk <= 7).
- * Larger requests return POETX_E_WORKSPACE without queueing anything.  The
+ * that loads it until the process exits.  It fits the build that runs:
+ * POETX_BF16 with b = 256 (one block per pair of SMs) takes 128 KiB per block
+ * plus 384 KiB per pair used, so nblk <= 47 on a 148-SM B200; the other
+ * builds take Q, S and H in fp32, nblk*b*b <= ~2.09e6 elements (b = 512:
+ * nblk <= 7; fp32 b = 64: nblk <= 511).  Larger requests return
+ * POETX_E_WORKSPACE without queueing anything.  The
  * first call on a device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current; make that first call
  * before any stream capture.  All calls share the one array and its contents
@@ -165,12 +189,13 @@ poetx_status poetx_cnp_backward(int32_t nblk, int32_t b, const float* q, const f
  * frame) for the backward; pass NULL for inference.  xg_save [T][m] (dtype,
  * nullable) receives Xg = x Psi_R^T, which spares the backward a gather of x.
  * Uses layer->GR/GP as last built by poetx_cnp_build.  T = 0 is a no-op.
- * bf16 layers with T > n apply Diag(G_R) to the weight rows instead of the
- * token rows (Y = Xg (W Diag(G_R)^T)^T, same product, rounded once at W_R
- * instead of at U).  With y_save == xg_save == NULL (inference) and
- * T > 6nm/(2m+4n), bf16 layers fold the whole layer into one natural-frame
- * weight and compute z = x W_eff^T as a single GEMM (same product, rounded
- * at the folded weights instead of at the activations). */
+ * With layer->fold == 0 every step acts on the token rows.  With
+ * POETX_FOLD_R, bf16 layers with T > n apply Diag(G_R) to the weight rows
+ * instead (Y = Xg (W Diag(G_R)^T)^T, same product, rounded once at W_R
+ * instead of at U).  With POETX_FOLD_WEIGHT_CENTRIC, y_save == xg_save ==
+ * NULL (inference) and T > 6nm/(2m+4n), bf16 layers fold the whole layer into
+ * one natural-frame weight and compute z = x W_eff^T as a single GEMM (same
+ * product, rounded at the folded weights instead of at the activations). */
 poetx_status poetx_forward(const poetx_layer* layer, int64_t T, const void* x, void* z, void* y_save,
                            void* xg_save, void* ws, size_t ws_bytes, void* stream);
 
@@ -183,9 +208,11 @@ poetx_status poetx_forward(const poetx_layer* layer, int64_t T, const void* x, v
  * write-up's section "三种变体", which keeps no [T][n] activation); its
  * workspace is then poetx_backward_recompute_workspace_bytes.  W0 is frozen,
  * so no dW0.  The dq sums over tokens use a fixed split and order
- * (deterministic for a given shape).  bf16 layers with T > m form
- * dU = dV (Diag(G_P)^T W) instead of (dV Diag(G_P)^T) W (same product,
- * rounded once at the folded weight instead of at dY). */
+ * (deterministic for a given shape).  With POETX_FOLD_P, bf16 layers with
+ * T > m form dU = dV (Diag(G_P)^T W) instead of (dV Diag(G_P)^T) W (same
+ * product, rounded once at the folded weight instead of at dY).  The
+ * recomputing backward takes the forward's fold decisions, so its Y is the
+ * forward's bit for bit. */
 poetx_status poetx_backward(const poetx_layer* layer, int64_t T, const void* x, const void* y_save,
                             const void* xg_save, const void* dz, void* dx, float* dqR, float* dqP,
                             int32_t accumulate, void* ws, size_t ws_bytes, void* stream);
@@ -216,6 +243,17 @@ poetx_status poetx_merge(const poetx_layer* layer, const int32_t* new_permR, con
  * 0..len-1, else 0. */
 poetx_status poetx_check_perm(const int32_t* perm, int32_t len, int32_t* d_ok, void* ws, size_t ws_bytes,
                               void* stream);
+
+/* Self-test of the failure path (no counterpart in the write-up): queues one
+ * warp that waits on an mbarrier no thread arrives on, through the bounded
+ * wait every kernel of the library uses, but with a limit of limit_us
+ * microseconds (1..1000000) instead of 4 s.  The wait gives up, records bit 1
+ * in the sticky device error word (read it with poetx_device_error) and the
+ * kernel returns, leaving the context usable for further calls.  d_out
+ * (device, 2 x uint64, 8-byte aligned): [0] = 1 if the wait ended by an
+ * arrival (never expected), [1] = nanoseconds waited.  POETX_E_ARG for a
+ * limit out of range or a NULL d_out. */
+poetx_status poetx_selftest_wait_timeout(uint32_t limit_us, unsigned long long* d_out, void* stream);
 
 /* POET-XQ storage of the frozen weight (write-up section "POET-XQ"): the
  * base weight is kept quantized and dequantized at run time.  The pages fix no

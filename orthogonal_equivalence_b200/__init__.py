@@ -21,6 +21,11 @@ LIB_PATH = os.path.join(_HERE, "libpoetx_debug.so" if os.environ.get("POETX_DEBU
 
 POETX_FP32 = 0
 POETX_BF16 = 1
+# poetx_layer.fold bits (0 = the input-centric evaluation everywhere)
+POETX_FOLD_R = 1
+POETX_FOLD_P = 2
+POETX_FOLD_WEIGHT_CENTRIC = 4
+POETX_FOLD_ALL = 7
 
 STATUS_NAMES = {0: "POETX_OK", 1: "POETX_E_ARG", 2: "POETX_E_SHAPE", 3: "POETX_E_DTYPE", 4: "POETX_E_ALIGN",
                 5: "POETX_E_WORKSPACE", 6: "POETX_E_ARCH", 7: "POETX_E_CUDA"}
@@ -35,7 +40,8 @@ class PoetxError(RuntimeError):
 class poetx_layer(ctypes.Structure):
     _fields_ = [("m", ctypes.c_int32), ("n", ctypes.c_int32), ("b", ctypes.c_int32), ("dtype", ctypes.c_int32),
                 ("W", ctypes.c_void_p), ("permR", ctypes.c_void_p), ("permP", ctypes.c_void_p),
-                ("qR", ctypes.c_void_p), ("qP", ctypes.c_void_p), ("GR", ctypes.c_void_p), ("GP", ctypes.c_void_p)]
+                ("qR", ctypes.c_void_p), ("qP", ctypes.c_void_p), ("GR", ctypes.c_void_p), ("GP", ctypes.c_void_p),
+                ("fold", ctypes.c_int32)]
 
 
 _VP, _I32, _I64, _SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
@@ -68,6 +74,7 @@ SIGNATURES = {
     "poetx_check_perm": (ctypes.c_int, [_VP, _I32, _VP, _VP, _SZ, _VP]),
     "poetx_weight_quantize": (ctypes.c_int, [_I32, _I32, _VP, _I32, _VP, _VP, _VP]),
     "poetx_weight_dequantize": (ctypes.c_int, [_I32, _I32, _VP, _VP, _I32, _VP, _VP]),
+    "poetx_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_uint32, _VP, _VP]),
     "poetx_adamw_step": (ctypes.c_int, [_I64, _VP, _VP, _VP, _VP, ctypes.c_float, ctypes.c_float, ctypes.c_float,
                                         ctypes.c_float, ctypes.c_float, _I32, _VP]),
     "poetx_profile_stage_count": (_I32, []),
@@ -118,8 +125,9 @@ def _check(status: int, where: str) -> None:
         raise PoetxError(status, where, lib().poetx_status_string(status).decode())
 
 
-def make_layer(m: int, n: int, b: int, dtype: int, W, permR, permP, qR, qP, GR, GP) -> poetx_layer:
-    return poetx_layer(m, n, b, dtype, _ptr(W), _ptr(permR), _ptr(permP), _ptr(qR), _ptr(qP), _ptr(GR), _ptr(GP))
+def make_layer(m: int, n: int, b: int, dtype: int, W, permR, permP, qR, qP, GR, GP, fold: int = 0) -> poetx_layer:
+    return poetx_layer(m, n, b, dtype, _ptr(W), _ptr(permR), _ptr(permP), _ptr(qR), _ptr(qP), _ptr(GR), _ptr(GP),
+                       fold)
 
 
 # ---------------------------------------------------------------- C calls, same names
@@ -251,6 +259,13 @@ def poetx_adamw_step(n: int, q, grad, m1, m2, lr: float, beta1: float, beta2: fl
                      weight_decay: float, step: int, stream=None) -> None:
     _check(lib().poetx_adamw_step(n, _ptr(q), _ptr(grad), _ptr(m1), _ptr(m2), lr, beta1, beta2, eps, weight_decay,
                                   step, _stream(stream)), "poetx_adamw_step")
+
+
+def poetx_selftest_wait_timeout(limit_us: int, d_out, stream=None) -> None:
+    """Queue the failure-path self-test: a bounded wait nobody satisfies gives
+    up after limit_us and records bit 1 in the device error word; d_out is a
+    device int64 tensor of 2 entries ([0] arrived, [1] ns waited)."""
+    _check(lib().poetx_selftest_wait_timeout(limit_us, _ptr(d_out), _stream(stream)), "poetx_selftest_wait_timeout")
 
 
 def poetx_profile_begin() -> None:

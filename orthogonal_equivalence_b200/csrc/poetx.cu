@@ -107,6 +107,7 @@ poetx_status check_layer(const poetx_layer* L) {
   POETX_TRY(check_dtype_b(L->dtype, L->b));
   if (L->m <= 0 || L->n <= 0 || L->m % L->b != 0 || L->n % L->b != 0) return POETX_E_SHAPE;
   if (L->m > kMaxM || L->n > max_n(L->dtype)) return POETX_E_SHAPE;
+  if (L->fold & ~POETX_FOLD_ALL) return POETX_E_ARG;
   const void* ptrs[] = {L->W, L->permR, L->permP, L->qR, L->qP, L->GR, L->GP};
   for (const void* p : ptrs) {
     if (!p) return POETX_E_ARG;
@@ -670,18 +671,23 @@ cudaError_t launch_bdg(const void* D, const void* X, const void* G, void* O, flo
   return cudaGetLastError();
 }
 
-// Y = (Xg Diag(G_R)) W~^T for T token rows.  When T > n the R-side block
-// product is applied to the n rows of the weight instead of the T rows of
-// activations: W_R = W~ Diag(G_R)^T ([n][m], one weight-sized pass), then
-// Y = Xg W_R^T, which skips the [T][m] intermediate U.  `scratch` holds U
-// ([T][m]) or W_R ([n][m], smaller when T > n).  The choice depends only on
-// (layer, T), so a recomputing backward gets the forward's Y bit for bit.
-bool fold_r_into_weight(const poetx_layer& L, int64_t T) { return L.dtype == POETX_BF16 && T > L.n; }
+// Y = (Xg Diag(G_R)) W~^T for T token rows.  With POETX_FOLD_R and T > n
+// the R-side block product is applied to the n rows of the weight instead of
+// the T rows of activations: W_R = W~ Diag(G_R)^T ([n][m], one weight-sized
+// pass), then Y = Xg W_R^T, which skips the [T][m] intermediate U.
+// `scratch` holds U ([T][m]) or W_R ([n][m], smaller when T > n).  The choice
+// depends only on (layer, T), so a recomputing backward gets the forward's Y
+// bit for bit.  Without the flag (the default) the layer stays input-centric.
+bool fold_r_into_weight(const poetx_layer& L, int64_t T) {
+  return (L.fold & POETX_FOLD_R) && L.dtype == POETX_BF16 && T > L.n;
+}
 
-// Backward P side: dU = dV (Diag(G_P)^T W~) instead of (dV Diag(G_P)^T) W~
-// when T > m (the [n][m] folded weight is smaller than the [T][n] dY it
-// replaces, and fits in the dY buffer).
-bool fold_p_into_weight(const poetx_layer& L, int64_t T) { return L.dtype == POETX_BF16 && T > L.m; }
+// Backward P side, with POETX_FOLD_P: dU = dV (Diag(G_P)^T W~) instead of
+// (dV Diag(G_P)^T) W~ when T > m (the [n][m] folded weight is smaller than
+// the [T][n] dY it replaces, and fits in the dY buffer).
+bool fold_p_into_weight(const poetx_layer& L, int64_t T) {
+  return (L.fold & POETX_FOLD_P) && L.dtype == POETX_BF16 && T > L.m;
+}
 
 // Wout = Diag(G_P)^T Win over the n/b row blocks of an [n][m] weight:
 // Wout[bj + c][i'] = sum_j' G_Pj[j'][c] Win[bj + j'][i'] (one batched GEMM).
@@ -721,14 +727,16 @@ cudaError_t fold_p_rows(const poetx_layer& L, const void* Win, void* Wout, cudaS
   return cudaSuccess;
 }
 
-// With nothing saved (inference, or a backward that recomputes), a forward
-// of T > 6nm / (2m + 4n) rows is cheaper as one GEMM with the whole layer
+// With nothing saved (inference, or a backward that recomputes) and
+// POETX_FOLD_WEIGHT_CENTRIC, a forward of T > 6nm / (2m + 4n) rows is cheaper
+// as one GEMM with the whole layer
 // folded into the weight in the natural frames,
 //   z = x W_eff^T,  W_eff = Psi_P^T Diag(G_P)^T W~ Diag(G_R)^T Psi_R,
 // than as gather, block products and scatter over the token rows (three
 // weight-sized passes instead of 2m + 4n activation columns).
 bool weight_centric_forward(const poetx_layer& L, int64_t T) {
-  return L.dtype == POETX_BF16 && T * (2 * int64_t(L.m) + 4 * int64_t(L.n)) > 6 * int64_t(L.n) * L.m;
+  return (L.fold & POETX_FOLD_WEIGHT_CENTRIC) && L.dtype == POETX_BF16 &&
+         T * (2 * int64_t(L.m) + 4 * int64_t(L.n)) > 6 * int64_t(L.n) * L.m;
 }
 
 cudaError_t y_from_xg(const poetx_layer& L, int64_t T, const void* Xg, void* Y, void* scratch, cudaStream_t st,
@@ -968,7 +976,7 @@ const char* poetx_status_string(int status) {
   }
 }
 
-int32_t poetx_version(void) { return 10000; }
+int32_t poetx_version(void) { return 10100; }
 
 poetx_status poetx_device_error(uint32_t* code) {
   if (!code) return POETX_E_ARG;
@@ -1188,8 +1196,8 @@ poetx_status poetx_forward(const poetx_layer* layer, int64_t T, const void* x, v
   void* Y = y_save ? y_save : Yw;
   // Xg = x Psi_R^T  (columns gathered into the Psi_R frame)
   PROFILED(ST_PERMUTE, st, POETX_CUDA(permute_dt(L.dtype, x, Xg, T, L.m, L.permR, 0, st, dev)));
-  // Y = (Xg Diag(G_R)) W~^T  (W~ = Psi_R W0 Psi_P^T stored [n][m]); U in `U`, or
-  // the weight with G_R folded in when T > n
+  // Y = (Xg Diag(G_R)) W~^T  (W~ = Psi_R W0 Psi_P^T stored [n][m]); U in `U`, or,
+  // with POETX_FOLD_R and T > n, the weight with G_R folded in
   POETX_CUDA(y_from_xg(L, T, Xg, Y, U, st, dev));
   // V_j = Y_j G_Pj
   PROFILED(ST_BLOCKDIAG, st, POETX_CUDA(launch_gemm(blockdiag_desc(Y, et, T, L.n, L.b, L.GP, false, V, et), tc_path, st, dev)));
@@ -1264,8 +1272,8 @@ static poetx_status backward_impl(const poetx_layer* layer, int64_t T, const voi
   void* dV = bufA;
   PROFILED(ST_PERMUTE, st, POETX_CUDA(permute_dt(L.dtype, dz, dV, T, L.n, L.permP, 0, st, dev)));
   // dY_j = dV_j G_Pj^T and dG_Pj = Y_j^T dV_j (split over tokens): one kernel
-  // reading dV once (b = 256 bf16), else two GEMMs.  When T > m (bf16) dY is
-  // not formed at all: G_P is folded into the weight (W_P = Diag(G_P)^T W~,
+  // reading dV once (b = 256 bf16), else two GEMMs.  With POETX_FOLD_P and
+  // T > m (bf16) dY is not formed at all: G_P is folded into the weight (W_P = Diag(G_P)^T W~,
   // [n][m], one weight-sized pass) and dU = dV W_P below, so only the dG
   // product reads dV here.
   void* dY = bufB;
@@ -1552,7 +1560,10 @@ int32_t poetx_profile_records(int32_t* stages, float* ms, int32_t max_records) {
 // and forbids allocations afterwards.  For them poetx_cnp_build_fixed takes
 // its scratch (Q, S and H for every block) from this file-scope device array
 // instead of a caller workspace.  The array is kFixedScratchBytes on every
-// GPU that loads the library, for the life of the process.  Host code must
+// GPU that loads the library, for the life of the process: b = 256 bf16
+// builds of up to 47 blocks (the pair kernel takes 128 KiB per block plus
+// three per pair of SMs), other builds of up to ~2.09e6 fp32 elements of Q
+// (b = 512: 7 blocks).  Host code must
 // not hand the symbol itself to a kernel (on the host it only names the
 // array); the device address comes from cudaGetSymbolAddress, looked up once
 // per device on that device's first call.
@@ -1586,15 +1597,55 @@ extern "C" poetx_status poetx_cnp_build_fixed(int32_t nblk, int32_t b, const flo
   if (nblk == 0) return POETX_OK;
   POETX_TRY(check_ptr(q));
   POETX_TRY(check_ptr(G));
-  const size_t need = kAlign + 3 * cnp_units(nblk, b);
-  if (need > kFixedScratchBytes) return POETX_E_WORKSPACE;  // too many blocks for the fixed scratch
   int dev;
   POETX_TRY(current_device(&dev));
+  // the scratch the build will carve: the fused pair kernel's bf16 operand
+  // region (b = 256 bf16), else Q, S and H in fp32 for every block; requests
+  // that do not fit are refused before anything is queued
+  const size_t need = kAlign + (use_pair_cnp(b, dtype) ? cnp_pair_bytes(nblk, false, false, dev)
+                                                       : 3 * cnp_units(nblk, b));
+  if (need > kFixedScratchBytes) return POETX_E_WORKSPACE;  // too many blocks for the fixed scratch
   void* scratch = nullptr;
   POETX_TRY(fixed_scratch(dev, &scratch));
-  // Q, S and H are written in full before they are read: nothing to clear.
+  // Every scratch matrix (Q, S, H, or the pair kernel's bf16 operands) is
+  // written in full before it is read: nothing to clear.
   Carver c(scratch, kFixedScratchBytes);
   return cnp_build2(b, dtype, q, nblk, G, nullptr, 0, nullptr, c, static_cast<cudaStream_t>(stream), dev);
+}
+
+// ---------------------------------------------------------------- failure-path self-test
+// One warp waits on an mbarrier that no thread ever arrives on, through the
+// same bounded wait the GEMM and copy kernels use, with a short limit: the
+// wait gives up, records DERR_GEMM_WAIT in the sticky error word and the
+// kernel returns normally.  No copy, MMA or TMEM allocation is involved, so
+// nothing is left in flight.  out[0] = 1 if the wait ended by an arrival
+// (never expected), out[1] = nanoseconds waited.
+namespace {
+__global__ void stalled_wait_kernel(uint64_t limit_ns, unsigned long long* out) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint64_t t0 = global_ns();
+    const bool arrived = mbar_wait_for(smem_u32(&bar), 0, DERR_GEMM_WAIT, limit_ns);
+    out[0] = arrived ? 1ull : 0ull;
+    out[1] = global_ns() - t0;
+  }
+}
+}  // namespace
+
+extern "C" poetx_status poetx_selftest_wait_timeout(uint32_t limit_us, unsigned long long* d_out, void* stream) {
+  if (limit_us < 1 || limit_us > 1000000) return POETX_E_ARG;
+  if (!d_out) return POETX_E_ARG;
+  if (reinterpret_cast<uintptr_t>(d_out) & 7u) return POETX_E_ALIGN;
+  int dev;
+  POETX_TRY(current_device(&dev));
+  stalled_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(uint64_t(limit_us) * 1000ull, d_out);
+  POETX_CUDA(cudaGetLastError());
+  return POETX_OK;
 }
 
 // ---------------------------------------------------------------- POET-XQ weight storage

@@ -91,18 +91,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Wait until the phase with the given parity has completed.  Returns false
-// (and records `code`) if that has not happened within POETX_WAIT_NS.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned int code) {
+// (and records `code`) if that has not happened within limit_ns of global time.
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, unsigned int code, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   uint32_t spins = 0;
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((++spins & 255u) == 0u && global_ns() - t0 > POETX_WAIT_NS) {
+    if ((++spins & 255u) == 0u && global_ns() - t0 > limit_ns) {
       record_error(code);
       return false;
     }
   }
+}
+
+// The kernels' wait: bounded by POETX_WAIT_NS.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned int code) {
+  return mbar_wait_for(bar, parity, code, POETX_WAIT_NS);
 }
 
 // ---------------------------------------------------------------- TMA (no multicast)

@@ -12,7 +12,7 @@ from typing import NamedTuple, Optional, Tuple
 
 import torch
 
-from . import (POETX_BF16, POETX_FP32, make_layer, poetx_backward, poetx_backward_dG,
+from . import (POETX_BF16, POETX_FOLD_ALL, POETX_FP32, make_layer, poetx_backward, poetx_backward_dG,
                poetx_backward_recompute_workspace_bytes, poetx_backward_workspace_bytes, poetx_cnp_backward,
                poetx_cnp_workspace_bytes,
                poetx_forward, poetx_forward_workspace_bytes, poetx_frame_export, poetx_frame_import,
@@ -47,11 +47,18 @@ class Saved(NamedTuple):
 
 
 class PoetxLinear:
-    """One layer z = x R W0 P (x: [T][m], z: [T][n])."""
+    """One layer z = x R W0 P (x: [T][m], z: [T][n]).
 
-    def __init__(self, m: int, n: int, b: int, dtype: int, device="cuda"):
+    `fold` (POETX_FOLD_* bits, default 0) lets a bf16 layer apply a block
+    product to the weight instead of the token rows where that moves fewer
+    bytes; 0 keeps the write-up's input-centric evaluation everywhere."""
+
+    def __init__(self, m: int, n: int, b: int, dtype: int, device="cuda", fold: int = 0):
         if dtype not in _TORCH_DTYPE:
             raise ValueError("dtype must be POETX_BF16 or POETX_FP32")
+        if fold & ~POETX_FOLD_ALL:
+            raise ValueError("fold: unknown POETX_FOLD bits")
+        self.fold = fold
         self.m, self.n, self.b, self.dtype = m, n, b, dtype
         self.device = torch.device(device)
         td = _TORCH_DTYPE[dtype]
@@ -96,7 +103,7 @@ class PoetxLinear:
 
     def abi(self):
         return make_layer(self.m, self.n, self.b, self.dtype, self.W, self.permR, self.permP, self.qR, self.qP,
-                          self.GR, self.GP)
+                          self.GR, self.GP, self.fold)
 
     def workspace(self, kind: str, nbytes: int) -> torch.Tensor:
         ws = self._ws.get(kind)

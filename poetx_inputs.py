@@ -84,6 +84,15 @@ CONFIGS = {
 }
 
 
+# Triangle scale of the parity cases that must see every term of the
+# Cayley-Neumann block: sigma per b with ||Q||_2 ~= 0.75-0.8 (the spectral
+# norm of a b x b skew Gaussian is about 2 sigma sqrt(b)).  At the workloads'
+# own scale (0.01, or 0.005 at b = 512) the Q^4 term moves G by less than the
+# bf16 bar; here leaving out Q^4, or 2Q^3, moves G, dq and the layer's
+# outputs by at least 3x the bar (a CPU test checks this on the oracle).
+PARITY_SIGMA = {64: 0.05, 128: 0.035, 256: 0.025, 512: 0.018}
+
+
 def seed_of(cfg: Config, layer: int, tensor: str, merge_index: int = 0) -> int:
     return 1000 * cfg.cfg_id + 10 * layer + TENSOR_IDS[tensor] + 100 * merge_index
 

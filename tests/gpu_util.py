@@ -40,8 +40,8 @@ def poetx_dtype(dtype: str) -> int:
     return px.POETX_BF16 if dtype == "bf16" else px.POETX_FP32
 
 
-def make_layer(inp: pi.LayerInputs) -> px.PoetxLinear:
-    L = px.PoetxLinear(inp.m, inp.n, inp.b, poetx_dtype(inp.dtype))
+def make_layer(inp: pi.LayerInputs, fold: int = 0) -> px.PoetxLinear:
+    L = px.PoetxLinear(inp.m, inp.n, inp.b, poetx_dtype(inp.dtype), fold=fold)
     L.load(dev(inp.W0lin, inp.dtype), torch.from_numpy(inp.permR).cuda(), torch.from_numpy(inp.permP).cuda(),
            torch.from_numpy(inp.qR).cuda(), torch.from_numpy(inp.qP).cuda())
     return L

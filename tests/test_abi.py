@@ -48,11 +48,17 @@ def test_status_strings(lib):
     for code, name in px.STATUS_NAMES.items():
         assert px.poetx_status_string(code).startswith(name)
     assert "unknown" in px.poetx_status_string(99)
-    assert px.poetx_version() == 10000
+    assert px.poetx_version() == 10100
 
 
-def _layer(m=512, n=256, b=64, dtype=px.POETX_BF16, ptr=4096):
-    return px.poetx_layer(m, n, b, dtype, ptr, ptr, ptr, ptr, ptr, ptr, ptr)
+def _layer(m=512, n=256, b=64, dtype=px.POETX_BF16, ptr=4096, fold=0):
+    return px.poetx_layer(m, n, b, dtype, ptr, ptr, ptr, ptr, ptr, ptr, ptr, fold)
+
+
+def test_layer_struct_matches_the_header():
+    # the fold field follows the seven pointers: offset 72, struct size 80 (LP64)
+    assert px.poetx_layer.fold.offset == 16 + 7 * 8
+    assert ctypes.sizeof(px.poetx_layer) == 80
 
 
 def test_workspace_sizes_are_host_arithmetic(lib):
@@ -84,6 +90,9 @@ def test_validation_before_any_launch(lib):
     assert lib.poetx_forward(ctypes.byref(L), 10, 4096, 4096, None, None, 4096, 1 << 30, None) == 3  # E_DTYPE
     L = _layer(ptr=4100)
     assert lib.poetx_forward(ctypes.byref(L), 10, 4096, 4096, None, None, 4096, 1 << 30, None) == 4  # E_ALIGN
+    L = _layer(fold=8)
+    assert lib.poetx_forward(ctypes.byref(L), 10, 4096, 4096, None, None, 4096, 1 << 30, None) == 1  # fold bits
+    assert px.poetx_forward_workspace_bytes(L, 10) == 0
     L = _layer()
     assert lib.poetx_forward(ctypes.byref(L), -1, 4096, 4096, None, None, 4096, 1 << 30, None) == 1  # T < 0
     assert lib.poetx_forward(ctypes.byref(L), 2 ** 31, 4096, 4096, None, None, 4096, 1 << 30, None) == 2  # T big
@@ -112,6 +121,11 @@ def test_validation_before_any_launch(lib):
     # merge output may not overlap the stored weight
     assert lib.poetx_merge(ctypes.byref(L), 4096, 4096, 4096, 4096, 1 << 30, None) == 1
     assert lib.poetx_check_perm(4096, 0, 4096, 4096, 1 << 20, None) == 1
+    # failure-path self-test: limit out of range, NULL or misaligned output
+    assert lib.poetx_selftest_wait_timeout(0, 4096, None) == 1
+    assert lib.poetx_selftest_wait_timeout(1000001, 4096, None) == 1
+    assert lib.poetx_selftest_wait_timeout(1000, None, None) == 1
+    assert lib.poetx_selftest_wait_timeout(1000, 4100, None) == 4
 
 
 def test_no_device_call_fails_cleanly(lib):

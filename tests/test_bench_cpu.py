@@ -55,6 +55,61 @@ def test_two_rank_gradient_allreduce_and_max_timing():
         assert slowest == 11.5            # max over ranks of the per-rank times
 
 
+def _dp_worker(rank, world, port, out):
+    """Rank `rank` holds token rows rank::world of one small layer: it takes
+    the oracle's dG of its rows, sums dG across ranks with the bench's
+    overlapped all-reduce, and turns the sum into dq with the oracle's CNP
+    backward."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import torch.distributed as dist
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    import bench
+    import oracle
+    import poetx_inputs as pi
+    inp = pi.layer_inputs(pi.CONFIGS["attn3b"], 0, T=50, m=128, n=192, b=64, sigma_q=0.03)
+    rows = np.arange(rank, inp.T, world)
+    GR, GP = oracle.cnp_blocks(inp.qR, inp.b), oracle.cnp_blocks(inp.qP, inp.b)
+    _, dGR, dGP = oracle.backward(inp.x64[rows], inp.W0lin64.T, inp.permR, GR, inp.permP, GP, inp.dz64[rows])
+    flat = torch.from_numpy(np.concatenate([dGR.ravel(), dGP.ravel()]))
+    half = dGR.size
+    parts = [flat[:half], flat[half:]]          # one exchange per side, started back to back
+    bench.allreduce_finish([bench.allreduce_start(t) for t in parts])
+    dG = flat.numpy()
+    dqR = oracle.cnp_backward(inp.qR, inp.b, dG[:half].reshape(dGR.shape))
+    dqP = oracle.cnp_backward(inp.qP, inp.b, dG[half:].reshape(dGP.shape))
+    out.put((rank, dqR, dqP))
+    dist.destroy_process_group()
+
+
+def test_data_parallel_dG_sum_gives_the_all_token_dq():
+    """The data-parallel exchange of the bench: the CNP backward is linear in
+    dG and dG is a sum over tokens, so summing the per-rank dG (token rows
+    split across two ranks) and then running the CNP backward gives the dq of
+    all tokens on one rank."""
+    import numpy as np
+    sys.path.insert(0, ROOT)
+    import oracle
+    import poetx_inputs as pi
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_dp_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    inp = pi.layer_inputs(pi.CONFIGS["attn3b"], 0, T=50, m=128, n=192, b=64, sigma_q=0.03)
+    _, dqR, dqP = oracle.layer_backward(inp.x64, inp.W0lin64.T, inp.permR, inp.qR, inp.permP, inp.qP, inp.b,
+                                        inp.dz64)
+    for _, gR, gP in res:
+        np.testing.assert_allclose(gR, dqR, rtol=1e-11, atol=1e-12 * np.abs(dqR).max())
+        np.testing.assert_allclose(gP, dqP, rtol=1e-11, atol=1e-12 * np.abs(dqP).max())
+
+
 def test_reference_arm_json_contract():
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
                           "tiny", "--steps", "2", "--warmup", "3", "--ref-tokens", "16"],

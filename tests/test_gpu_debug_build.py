@@ -28,10 +28,13 @@ from gpu_util import dev, make_layer
 
 px.poetx_device_error()
 out = {}
-# a: P side with G_P folded, R side fused; b: both folds; c: P side fused (T <= m)
-for tag, (m, n, T) in {"a": (512, 1024, 1000), "b": (1024, 512, 2000), "c": (1024, 512, 700)}.items():
+# a: P side with G_P folded, R side fused; b: both folds; c: P side fused
+# (T <= m); d: input-centric with T > m, n (both sides fused)
+F = px.POETX_FOLD_ALL
+for tag, (m, n, T, fold) in {"a": (512, 1024, 1000, F), "b": (1024, 512, 2000, F), "c": (1024, 512, 700, F),
+                             "d": (1024, 512, 2000, 0)}.items():
     inp = pi.layer_inputs(pi.CONFIGS["block8b"], layer=0, T=T, m=m, n=n, b=256)
-    L = make_layer(inp)
+    L = make_layer(inp, fold)
     x, dz = dev(inp.x, "bf16"), dev(inp.dz, "bf16")
     z, saved = L.forward(x, save_xg=True)
     dx, dqR, dqP = L.backward(x, saved, dz)

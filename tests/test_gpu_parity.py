@@ -32,7 +32,10 @@ def library():
     assert px.poetx_device_error() == 0, "a kernel recorded a device error (timeout or bad index)"
 
 
-# (workload recipe, m, n, b, T); None = the workload's own size
+# (workload recipe, m, n, b, T[, fold]); None = the workload's own size.
+# Without a fold entry the layer is evaluated input-centrically (fold 0), also
+# where T > m, n; the cases with FOLD also take the weight-fold paths.
+FOLD = px.POETX_FOLD_ALL
 SMALL = [
     ("tiny", None, None, None, None),
     ("tiny", 192, 320, 64, 77),
@@ -43,13 +46,27 @@ SMALL = [
     ("block8b", 256, 768, 256, 1),
     ("block8b", 512, 1024, 256, 1000),   # >= 4 token tiles: block-resident G path
     ("down13b", 1024, 1536, 512, 777),
-    ("down13b", 1024, 512, 512, 2000),   # T > m, n: both weight folds at b = 512
-    ("attn3b", 256, 384, 128, 1000),     # T > m, n: both weight folds at b = 128
+    ("down13b", 1024, 512, 512, 2000),   # T > m, n, input-centric at b = 512
+    ("attn3b", 256, 384, 128, 1000),     # T > m, n, input-centric at b = 128
+    ("block8b", 512, 256, 256, 2000),    # T > m, n, input-centric at b = 256 (fused bdg on both sides)
+    ("down13b", 1024, 512, 512, 2000, FOLD),   # T > m, n: both weight folds at b = 512
+    ("attn3b", 256, 384, 128, 1000, FOLD),     # T > m, n: both weight folds at b = 128
+    ("block8b", 512, 256, 256, 2000, FOLD),    # T > m, n: both weight folds at b = 256
 ]
 
+# One layer case per b at the triangle scale where leaving out the Q^4 or the
+# 2Q^3 term of G misses the bf16 bar by >= 3x (tests/test_parity_sigma.py
+# proves it on the oracle for these shapes).
+SIGMA_LAYERS = [("block8b", 192, 320, 64, 300), ("attn3b", 256, 384, 128, 1000), ("attn3b", 512, 512, 256, 300),
+                ("down13b", 1024, 1536, 512, 130), ("block8b", 512, 256, 256, 2000, FOLD)]
 
-def _inputs(name, m, n, b, T, layer=0, **kw):
+
+def _inputs(name, m, n, b, T, *fold, layer=0, **kw):
     return pi.layer_inputs(pi.CONFIGS[name], layer=layer, T=T, m=m, n=n, b=b, **kw)
+
+
+def _fold(case):
+    return case[5] if len(case) > 5 else 0
 
 
 def _oracle_all(inp):
@@ -73,7 +90,7 @@ def _run(L, inp):
 @pytest.mark.parametrize("case", SMALL, ids=lambda c: "-".join(str(v) for v in c))
 def test_layer_forward_backward_parity(case):
     inp = _inputs(*case)
-    L = make_layer(inp)
+    L = make_layer(inp, _fold(case))
     z, _, dx, dqR, dqP = _run(L, inp)
     zo, dxo, dqRo, dqPo, _, _ = _oracle_all(inp)
     check(host64(z), zo, inp.dtype, "z")
@@ -82,11 +99,29 @@ def test_layer_forward_backward_parity(case):
     check(host64(dqP), dqPo, inp.dtype, "dqP")
 
 
-@pytest.mark.parametrize("dtype,b,nblk", [("fp32", 64, 8), ("bf16", 256, 5), ("bf16", 512, 3), ("bf16", 64, 9),
-                                          ("fp32", 6, 4)])
-def test_cnp_build_and_backward_parity(dtype, b, nblk):
+@pytest.mark.parametrize("case", SIGMA_LAYERS, ids=lambda c: "-".join(str(v) for v in c))
+def test_layer_parity_at_discriminating_sigma(case):
+    inp = _inputs(*case, sigma_q=pi.PARITY_SIGMA[case[3]])
+    L = make_layer(inp, _fold(case))
+    z, _, dx, dqR, dqP = _run(L, inp)
+    zo, dxo, dqRo, dqPo, _, _ = _oracle_all(inp)
+    check(host64(z), zo, inp.dtype, "z")
+    check(host64(dx), dxo, inp.dtype, "dx")
+    check(host64(dqR), dqRo, inp.dtype, "dqR")
+    check(host64(dqP), dqPo, inp.dtype, "dqP")
+
+
+# sigma None: the workloads' scale 0.01; "parity": pi.PARITY_SIGMA[b], where
+# every term of G shows through the bar
+@pytest.mark.parametrize("dtype,b,nblk,sigma", [("fp32", 64, 8, None), ("bf16", 256, 5, None),
+                                                ("bf16", 512, 3, None), ("bf16", 64, 9, None), ("fp32", 6, 4, None),
+                                                ("bf16", 256, 5, "parity"), ("bf16", 512, 3, "parity"),
+                                                ("bf16", 128, 4, "parity"), ("bf16", 64, 9, "parity"),
+                                                ("fp32", 64, 8, "parity")])
+def test_cnp_build_and_backward_parity(dtype, b, nblk, sigma):
     g = np.random.Generator(np.random.PCG64(1000 + b + nblk))
-    q = (g.standard_normal((nblk, b * (b - 1) // 2)) * 0.01).astype(np.float32)
+    scale = pi.PARITY_SIGMA[b] if sigma == "parity" else 0.01
+    q = (g.standard_normal((nblk, b * (b - 1) // 2)) * scale).astype(np.float32)
     dG = g.standard_normal((nblk, b, b)).astype(np.float32)
     pd = poetx_dtype(dtype)
     td = torch.bfloat16 if dtype == "bf16" else torch.float32
@@ -108,14 +143,15 @@ def test_cnp_build_and_backward_parity(dtype, b, nblk):
     check(host64(dq), 2 * dqo, dtype, "dq accumulated")
 
 
-def test_cnp_full_batch_of_the_8b_block():
+@pytest.mark.parametrize("sigma", [0.01, pi.PARITY_SIGMA[256]])
+def test_cnp_full_batch_of_the_8b_block(sigma):
     """The 8B block's batched CNP size (320 blocks of b = 256: several blocks
     per pair of SMs): build and backward on sampled blocks against the oracle,
     a sub-batch gives the same bits as the full batch, and accumulating adds
     exactly the plain result."""
     nblk, b = 320, 256
     g = np.random.Generator(np.random.PCG64(4242))
-    q = (g.standard_normal((nblk, b * (b - 1) // 2)) * 0.01).astype(np.float32)
+    q = (g.standard_normal((nblk, b * (b - 1) // 2)) * sigma).astype(np.float32)
     dG = g.standard_normal((nblk, b, b)).astype(np.float32)
     qd, dGd = torch.from_numpy(q).cuda(), torch.from_numpy(dG).cuda()
     G = torch.empty((nblk, b, b), dtype=torch.bfloat16, device="cuda")
@@ -188,12 +224,13 @@ def test_frame_import_export_bit_exact(dtype, m, n):
     assert np.array_equal(bits(back), inp.W0lin.view(np.uint16 if dtype == "bf16" else np.uint32))
 
 
-def _merge_check(inp, merge_index=1):
+def _merge_check(inp, merge_index=1, cfg=None, layer=0):
     L = make_layer(inp)
     x = dev(inp.x, inp.dtype)
     z_before, _ = L.forward(x, save=False)
-    newR, newP = pi.merge_perms(pi.CONFIGS["tiny"] if inp.dtype == "fp32" else pi.CONFIGS["down13b"], 0,
-                                merge_index, inp.m, inp.n)
+    if cfg is None:
+        cfg = pi.CONFIGS["tiny"] if inp.dtype == "fp32" else pi.CONFIGS["down13b"]
+    newR, newP = pi.merge_perms(cfg, layer, merge_index, inp.m, inp.n)
     L.merge(torch.from_numpy(newR).cuda(), torch.from_numpy(newP).cuda())
     W_nat = L.export_weight()
     torch.cuda.synchronize()
@@ -287,14 +324,16 @@ def test_saved_xg_backward_matches_regather(case):
 
 
 @pytest.mark.parametrize("case", [("block8b", 512, 256, 256, 2000), ("up8b", 256, 768, 256, 1500),
-                                  ("attn3b", 512, 512, 256, 300)], ids=lambda c: f"{c[0]}-{c[4]}")
+                                  ("attn3b", 512, 512, 256, 300), ("block8b", 512, 256, 256, 2000, FOLD),
+                                  ("up8b", 256, 768, 256, 1500, FOLD)], ids=lambda c: f"{c[0]}-{c[4]}-{_fold(c)}")
 def test_forward_without_saving(case):
     """A forward that saves nothing (inference, or the recomputing backward's
-    forward): above T = 6nm/(2m+4n) the whole layer is one GEMM with the
-    weight folded into the natural frames; z against the oracle and against
-    the forward that saves Y (which takes the token-row path)."""
+    forward): input-centric by default; with POETX_FOLD_WEIGHT_CENTRIC and
+    T above 6nm/(2m+4n) the whole layer is one GEMM with the weight folded
+    into the natural frames; z against the oracle and against the forward that
+    saves Y (which takes the token-row path)."""
     inp = _inputs(*case)
-    L = make_layer(inp)
+    L = make_layer(inp, _fold(case))
     x = dev(inp.x, inp.dtype)
     z_nosave, _ = L.forward(x, save=False)
     z_save, _ = L.forward(x)
@@ -305,13 +344,14 @@ def test_forward_without_saving(case):
 
 
 @pytest.mark.parametrize("case", [("up8b", 512, 1024, 256, 700), ("tiny", 192, 320, 64, 77),
-                                  ("block8b", 512, 256, 256, 600)],   # T > m, n: both weight folds
-                         ids=lambda c: f"{c[0]}-{c[4]}")
+                                  ("block8b", 512, 256, 256, 600),
+                                  ("block8b", 512, 256, 256, 600, FOLD)],   # T > m, n: both weight folds
+                         ids=lambda c: f"{c[0]}-{c[4]}-{_fold(c)}")
 def test_recomputing_backward_mem_variant(case):
     # the "mem" variant keeps nothing from the forward: the backward recomputes
     # Y from x and must match the saved-Y backward bit for bit
     inp = _inputs(*case)
-    L = make_layer(inp)
+    L = make_layer(inp, _fold(case))
     x, dz = dev(inp.x, inp.dtype), dev(inp.dz, inp.dtype)
     _, saved = L.forward(x)
     dx1, r1, p1 = L.backward(x, saved, dz)
@@ -527,3 +567,15 @@ def test_full_size_sampled_parity(name):
 def test_full_size_merge_down13b():
     inp = pi.layer_inputs(pi.CONFIGS["down13b"], 0, T=256)
     _merge_check(inp)
+
+
+def test_full_size_merge_of_all_block8b_linears():
+    """The merge step of the 8B block: each of its seven linears at full size
+    (q, k, v, o, gate, up, down) merged with its own new permutations; merged
+    weight against the oracle's R W0 P, q = 0, G = I, and z unchanged."""
+    cfg = pi.CONFIGS["block8b"]
+    for layer in range(len(cfg.layers)):
+        inp = pi.layer_inputs(cfg, layer, T=64)
+        L = _merge_check(inp, cfg=cfg, layer=layer)
+        del L
+        torch.cuda.empty_cache()
