@@ -9,6 +9,7 @@
 #pragma once
 
 #include <cstdint>
+#include <type_traits>
 #include <cuda_bf16.h>
 
 #include "ptx.cuh"
@@ -270,6 +271,122 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(const T* __restrict__
         for (int k = 0; k < V; ++k) pk.e[k] = srow[iv[k]];
       }
       reinterpret_cast<uint4*>(out + (r0 + rr) * cols + c0)[0] = pk.u;
+    }
+    __syncthreads();  // stage s may be refilled next iteration
+  }
+  if (!ok && threadIdx.x == 0) {
+    // let a copy still in flight land before the block exits
+    for (int s = 0; s < 2; ++s)
+      if (pending & (1u << s)) mbar_wait(smem_u32(&full_bar[s]), phase[s], DERR_PERM_WAIT);
+  }
+}
+
+// permute_rows_kernel with every thread's index entries held in registers.
+// The block gives each thread a fixed set of output vectors: with vpr =
+// cols / V vectors per row, thread t owns vectors t, t + 256, ... of every
+// row (vpr >= 256), or, when vpr < 256, vector t % vpr of rows t / vpr,
+// t / vpr + 256 / vpr, ... of each stage.  So a thread reads its (at most
+// MAXV) vectors of indices out of the shared table once, before the first
+// stage, instead of once per row: the random 2-byte reads of the staged rows
+// are the only shared-memory loads left in the loop.
+template <typename T, int MAXV>
+__global__ void __launch_bounds__(256) permute_rows_reg_kernel(const T* __restrict__ in, T* __restrict__ out,
+                                                               int64_t rows, int cols,
+                                                               const int32_t* __restrict__ map, int inverse,
+                                                               int rows_per_stage) {
+  extern __shared__ __align__(128) uint8_t sm_raw[];
+  __shared__ __align__(8) uint64_t full_bar[2];
+  constexpr int V = 16 / sizeof(T);
+  using IdxVec = typename std::conditional<V == 8, uint4, uint2>::type;  // V 16-bit indices
+  uint16_t* idx = reinterpret_cast<uint16_t*>(sm_raw);
+  const size_t idx_bytes = (static_cast<size_t>(cols) * 2 + 127) & ~size_t(127);
+  T* stage_base = reinterpret_cast<T*>(sm_raw + idx_bytes);
+  const int64_t stage_elems = static_cast<int64_t>(rows_per_stage) * cols;
+  const int64_t nchunks = (rows + rows_per_stage - 1) / rows_per_stage;
+  const int vpr = cols / V;
+  const int nthr = static_cast<int>(blockDim.x);
+  // this thread's vectors: columns (vec0 + k * nthr) * V for k < nvec, in rows
+  // row0, row0 + rstep, ... of each stage
+  const bool wide = vpr >= nthr;
+  const int rstep = wide ? 1 : nthr / vpr;
+  const int vec0 = wide ? static_cast<int>(threadIdx.x) : static_cast<int>(threadIdx.x) % vpr;
+  const int row0 = wide ? 0 : static_cast<int>(threadIdx.x) / vpr;
+  const bool active = wide || static_cast<int>(threadIdx.x) < rstep * vpr;
+  const int nvec = wide ? (vpr - vec0 + nthr - 1) / nthr : 1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&full_bar[0]), 1);
+    mbar_init(smem_u32(&full_bar[1]), 1);
+    fence_barrier_init();
+  }
+  if (inverse) {
+    // entries a non-bijective map never reaches stay 0 (in range)
+    for (int c = threadIdx.x; c < cols; c += blockDim.x) idx[c] = 0;
+    __syncthreads();
+  }
+  for (int c = threadIdx.x; c < cols; c += blockDim.x) {
+    const int m = map[c];
+    if (m < 0 || m >= cols) {
+      record_error(DERR_BAD_INDEX);
+      if (!inverse) idx[c] = 0;
+      continue;
+    }
+    if (inverse) idx[m] = static_cast<uint16_t>(c);
+    else idx[c] = static_cast<uint16_t>(m);
+  }
+  __syncthreads();
+  IdxVec myidx[MAXV];
+#pragma unroll
+  for (int k = 0; k < MAXV; ++k)
+    if (active && k < nvec) myidx[k] = *reinterpret_cast<const IdxVec*>(idx + (vec0 + k * nthr) * V);
+
+  uint32_t pending = 0;  // stages with a copy in flight (thread 0's view)
+  auto issue = [&](int64_t chunk, int s) {
+    const int64_t r0 = chunk * rows_per_stage;
+    const int64_t nr = rows - r0 < rows_per_stage ? rows - r0 : rows_per_stage;
+    const uint32_t bytes = static_cast<uint32_t>(nr * cols * sizeof(T));
+    const uint32_t bar = smem_u32(&full_bar[s]);
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    mbar_arrive_expect_tx(bar, bytes);
+    bulk_load(smem_u32(stage_base + s * stage_elems), in + r0 * cols, bytes, bar);
+    pending |= 1u << s;
+  };
+
+  int64_t chunk = blockIdx.x;
+  if (threadIdx.x == 0 && chunk < nchunks) issue(chunk, 0);
+  uint32_t phase[2] = {0u, 0u};
+  bool ok = true;
+  for (int it = 0; chunk < nchunks; chunk += gridDim.x, ++it) {
+    const int s = it & 1;
+    const int64_t next = chunk + gridDim.x;
+    if (threadIdx.x == 0 && next < nchunks) issue(next, s ^ 1);
+    ok = mbar_wait(smem_u32(&full_bar[s]), phase[s], DERR_PERM_WAIT);
+    if (ok) {
+      phase[s] ^= 1u;
+      pending &= ~(1u << s);
+    }
+    if (!__syncthreads_and(ok)) break;
+    const int64_t r0 = chunk * rows_per_stage;
+    const int nr = static_cast<int>(rows - r0 < rows_per_stage ? rows - r0 : rows_per_stage);
+    const T* st = stage_base + s * stage_elems;
+    if (active) {
+      for (int rr = row0; rr < nr; rr += rstep) {
+        const T* srow = st + static_cast<int64_t>(rr) * cols;
+        T* orow = out + (r0 + rr) * cols;
+#pragma unroll
+        for (int k = 0; k < MAXV; ++k) {
+          if (k < nvec) {
+            const uint16_t* iv = reinterpret_cast<const uint16_t*>(&myidx[k]);
+            union {
+              uint4 u;
+              T e[V];
+            } pk;
+#pragma unroll
+            for (int e = 0; e < V; ++e) pk.e[e] = srow[iv[e]];
+            reinterpret_cast<uint4*>(orow + (vec0 + k * nthr) * V)[0] = pk.u;
+          }
+        }
+      }
     }
     __syncthreads();  // stage s may be refilled next iteration
   }

@@ -332,13 +332,24 @@ cudaError_t permute_cols(const T* in, T* out, int64_t rows, int cols, const int3
     return inverse ? scatter(in, cols, out, cols, rows, rows, cols, map, nullptr, st, device)
                    : gather(in, cols, rows, out, cols, rows, cols, map, nullptr, st, device);
   }
-  cudaError_t e = allow_smem(permute_rows_kernel<T>, smem, &attr[device & 63]);
+  // each thread's index entries in registers when it owns at most kRegVecs
+  // 16-byte output vectors per row
+  constexpr int kRegVecs = 8;
+  const int vpr = cols / V;
+  const bool reg_idx = (vpr + 255) / 256 <= kRegVecs;
+  static bool attr_reg[64] = {false};
+  cudaError_t e = reg_idx ? allow_smem(permute_rows_reg_kernel<T, kRegVecs>, smem, &attr_reg[device & 63])
+                          : allow_smem(permute_rows_kernel<T>, smem, &attr[device & 63]);
   if (e != cudaSuccess) return e;
   const int per_sm = static_cast<int>((220 * 1024) / (smem + 1024));
   const int64_t chunks = (rows + rps - 1) / rps;
   int64_t g = int64_t(sm_count(device)) * (per_sm < 1 ? 1 : (per_sm > 8 ? 8 : per_sm));
   if (g > chunks) g = chunks;
-  permute_rows_kernel<T><<<static_cast<int>(g), 256, smem, st>>>(in, out, rows, cols, map, inverse, rps);
+  if (reg_idx)
+    permute_rows_reg_kernel<T, kRegVecs><<<static_cast<int>(g), 256, smem, st>>>(in, out, rows, cols, map, inverse,
+                                                                                 rps);
+  else
+    permute_rows_kernel<T><<<static_cast<int>(g), 256, smem, st>>>(in, out, rows, cols, map, inverse, rps);
   return cudaGetLastError();
 }
 
