@@ -260,11 +260,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           // is stored
           uint32_t w[BLK / 2];
 #pragma unroll
-          for (int c = 0; c < BLK / 32; ++c) {
-            float v[32];
-            tmem_ld_32cols(tl + 32 * c, v);
+          for (int c = 0; c < BLK / 64; ++c) {
+            float v[32], u[32];
+            tmem_ld_32cols_x2(tl + 64 * c, tl + 64 * c + 32, v, u);  // one round trip per 64 columns
 #pragma unroll
-            for (int i = 0; i < 16; ++i) w[16 * c + i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+            for (int i = 0; i < 16; ++i) w[32 * c + i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) w[32 * c + 16 + i] = pack_bf16x2(u[2 * i], u[2 * i + 1]);
           }
           tc_fence_before();
           __syncwarp();
@@ -300,12 +302,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       float* dst = p.part + ((int64_t(s) * p.nblk + j) * BLK + int(rank) * HALF + quarter * 32 + lane) * BLK;
 #pragma unroll 1
-      for (int c0 = 0; c0 < BLK; c0 += 32) {
-        float v[32];
-        tmem_ld_32cols(tl + BLK + c0, v);
+      for (int c0 = 0; c0 < BLK; c0 += 64) {
+        float v[32], v2[32];
+        tmem_ld_32cols_x2(tl + BLK + c0, tl + BLK + c0 + 32, v, v2);
         float4* d4 = reinterpret_cast<float4*>(dst + c0);
 #pragma unroll
         for (int u = 0; u < 8; ++u) d4[u] = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) d4[8 + u] = make_float4(v2[4 * u], v2[4 * u + 1], v2[4 * u + 2], v2[4 * u + 3]);
       }
       tc_fence_before();
       __syncwarp();

@@ -394,50 +394,66 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           tc_fence_after();
           const uint32_t t0 = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
           float v0[32], v1[32], w[32];
-          for (int c0 = 0; c0 < BLK; c0 += 32) {
+          // 64 columns per step: the TMEM loads of a step share one round trip
+          for (int c0 = 0; c0 < BLK; c0 += 64) {
             const uint32_t tileA = smem_base + (c0 >> 6) * STAGE_BYTES, tileB = tileA + TILE_BYTES;
             if (ph == 1) {
               // S = -acc0;  H = S + 2Q (build) or H^T = S - 2Q (backward); Q from P1's A tiles
-              tmem_ld_32cols(t0 + c0, v0);
-              tile_row_bf16x32(tileA, lrow, c0, w);
+              float a1[32];
+              tmem_ld_32cols_x2(t0 + c0, t0 + c0 + 32, v0, a1);
               const float sgn = p.backward ? -2.f : 2.f;
 #pragma unroll
-              for (int e = 0; e < 32; ++e) {
-                v0[e] = -v0[e];
-                v1[e] = v0[e] + sgn * w[e];
+              for (int h = 0; h < 2; ++h) {
+                const int cc = c0 + 32 * h;
+                float* a = h ? a1 : v0;
+                tile_row_bf16x32(tileA, lrow, cc, w);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                  a[e] = -a[e];
+                  v1[e] = a[e] + sgn * w[e];
+                }
+                store_bf16x32(matp(slot0 + KS) + row * BLK + cc, a);
+                store_bf16x32(matp(slot0 + KH) + row * BLK + cc, v1);
               }
-              store_bf16x32(matp(slot0 + KS) + row * BLK + c0, v0);
-              store_bf16x32(matp(slot0 + KH) + row * BLK + c0, v1);
             } else if (!p.backward) {
               // G = I + 2Q + 2S + acc1, 2Q = H - S from P2's A (H) and B (S) tiles, S = -acc0
-              tmem_ld_32cols(t0 + c0, v0);
-              tmem_ld_32cols(t0 + BLK + c0, v1);
-              tile_row_bf16x32(tileA, lrow, c0, w);
-              float sb[32];
-              tile_row_bf16x32(tileB, lrow, c0, sb);
+#pragma unroll 1
+              for (int h = 0; h < 2; ++h) {
+                const int cc = c0 + 32 * h;
+                tmem_ld_32cols_x2(t0 + cc, t0 + BLK + cc, v0, v1);
+                tile_row_bf16x32(tileA, lrow, cc, w);
+                float sb[32];
+                tile_row_bf16x32(tileB, lrow, cc, sb);
 #pragma unroll
-              for (int e = 0; e < 32; ++e)
-                v1[e] = ((c0 + e == row ? 1.f : 0.f) + (w[e] - sb[e])) + (-2.f * v0[e]) + v1[e];
-              __nv_bfloat16* G = static_cast<__nv_bfloat16*>(sg.out[s]) + int64_t(lt) * BLK * BLK;
-              store_bf16x32(G + row * BLK + c0, v1);
+                for (int e = 0; e < 32; ++e)
+                  v1[e] = ((cc + e == row ? 1.f : 0.f) + (w[e] - sb[e])) + (-2.f * v0[e]) + v1[e];
+                __nv_bfloat16* G = static_cast<__nv_bfloat16*>(sg.out[s]) + int64_t(lt) * BLK * BLK;
+                store_bf16x32(G + row * BLK + cc, v1);
+              }
             } else if (ph == 2) {
               // dS = 2dG + acc0 + acc1 (a bf16 operand; dG from P2's A tiles); acc1 <- 2 acc1
-              tmem_ld_32cols(t0 + c0, v0);
-              tmem_ld_32cols(t0 + BLK + c0, v1);
-              tile_row_bf16x32(tileA, lrow, c0, w);
+#pragma unroll 1
+              for (int h = 0; h < 2; ++h) {
+                const int cc = c0 + 32 * h;
+                tmem_ld_32cols_x2(t0 + cc, t0 + BLK + cc, v0, v1);
+                tile_row_bf16x32(tileA, lrow, cc, w);
 #pragma unroll
-              for (int e = 0; e < 32; ++e) {
-                v0[e] = (2.f * w[e] + v0[e]) + v1[e];
-                v1[e] = 2.f * v1[e];
+                for (int e = 0; e < 32; ++e) {
+                  v0[e] = (2.f * w[e] + v0[e]) + v1[e];
+                  v1[e] = 2.f * v1[e];
+                }
+                store_bf16x32(matp(slot0 + KDS) + row * BLK + cc, v0);
+                tmem_st_32cols(t0 + BLK + cc, v1);
               }
-              store_bf16x32(matp(slot0 + KDS) + row * BLK + c0, v0);
-              tmem_st_32cols(t0 + BLK + c0, v1);
             } else {
               // acc1 = dA - 2dG for the fold (padded rows: conflict-free transposed reads)
-              tmem_ld_32cols(t0 + BLK + c0, v0);
+              tmem_ld_32cols_x2(t0 + BLK + c0, t0 + BLK + c0 + 32, v0, v1);
               float* d = dAs + lrow * DA_LD + c0;
 #pragma unroll
-              for (int e = 0; e < 32; ++e) d[e] = v0[e];
+              for (int e = 0; e < 32; ++e) {
+                d[e] = v0[e];
+                d[32 + e] = v1[e];
+              }
             }
           }
         }

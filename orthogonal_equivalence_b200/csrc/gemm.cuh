@@ -455,13 +455,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int c0 = 0; c0 < BN; c0 += cho) {
         uint32_t w[32];  // one 128-byte output row of this lane
         if (e.c_et == ET_BF16) {
-          float v[32];
-          tmem_ld_32cols(tl + c0, v);
+          float v[32], u[32];
+          tmem_ld_32cols_x2(tl + c0, tl + c0 + 32, v, u);
 #pragma unroll
           for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(e.alpha * v[2 * i], e.alpha * v[2 * i + 1]);
-          tmem_ld_32cols(tl + c0 + 32, v);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) w[16 + i] = pack_bf16x2(e.alpha * v[2 * i], e.alpha * v[2 * i + 1]);
+          for (int i = 0; i < 16; ++i) w[16 + i] = pack_bf16x2(e.alpha * u[2 * i], e.alpha * u[2 * i + 1]);
         } else {
           float v[32];
           tmem_ld_32cols(tl + c0, v);
