@@ -259,7 +259,7 @@ int grid_for(int64_t n, int threads, int device) {
 
 template <typename K>
 cudaError_t allow_smem(K kernel, size_t bytes, bool* done) {
-  if (bytes <= 48 * 1024 || *done) return cudaSuccess;
+  if (bytes + 1024 <= 48 * 1024 || *done) return cudaSuccess;  // (static shared memory counts too)
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
   if (e == cudaSuccess) *done = true;
   return e;
