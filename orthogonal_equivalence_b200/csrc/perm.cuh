@@ -293,15 +293,18 @@ template <typename T, int MAXV>
 __global__ void __launch_bounds__(256) permute_rows_reg_kernel(const T* __restrict__ in, T* __restrict__ out,
                                                                int64_t rows, int cols,
                                                                const int32_t* __restrict__ map, int inverse,
-                                                               int rows_per_stage) {
+                                                               int rows_per_stage, int idx_in_stage) {
   extern __shared__ __align__(128) uint8_t sm_raw[];
   __shared__ __align__(8) uint64_t full_bar[2];
   constexpr int V = 16 / sizeof(T);
   using IdxVec = typename std::conditional<V == 8, uint4, uint2>::type;  // V 16-bit indices
-  uint16_t* idx = reinterpret_cast<uint16_t*>(sm_raw);
   const size_t idx_bytes = (static_cast<size_t>(cols) * 2 + 127) & ~size_t(127);
-  T* stage_base = reinterpret_cast<T*>(sm_raw + idx_bytes);
+  // the index table is only read before the first stage lands: with
+  // idx_in_stage it lives in stage 1, which is first filled after that
+  T* stage_base = reinterpret_cast<T*>(sm_raw + (idx_in_stage ? 0 : idx_bytes));
   const int64_t stage_elems = static_cast<int64_t>(rows_per_stage) * cols;
+  uint16_t* idx = idx_in_stage ? reinterpret_cast<uint16_t*>(stage_base + stage_elems)
+                               : reinterpret_cast<uint16_t*>(sm_raw);
   const int64_t nchunks = (rows + rows_per_stage - 1) / rows_per_stage;
   const int vpr = cols / V;
   const int nthr = static_cast<int>(blockDim.x);
@@ -339,6 +342,7 @@ __global__ void __launch_bounds__(256) permute_rows_reg_kernel(const T* __restri
 #pragma unroll
   for (int k = 0; k < MAXV; ++k)
     if (active && k < nvec) myidx[k] = *reinterpret_cast<const IdxVec*>(idx + (vec0 + k * nthr) * V);
+  __syncthreads();  // every thread has its indices before stage 1 may be overwritten
 
   uint32_t pending = 0;  // stages with a copy in flight (thread 0's view)
   auto issue = [&](int64_t chunk, int s) {

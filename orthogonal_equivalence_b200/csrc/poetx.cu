@@ -326,7 +326,7 @@ cudaError_t permute_cols(const T* in, T* out, int64_t rows, int cols, const int3
   if (rps < 1) rps = 1;
   if (rps > 64) rps = 64;
   const size_t idx_bytes = (size_t(cols) * 2 + 127) & ~size_t(127);
-  const size_t smem = idx_bytes + 2 * size_t(rps) * row_bytes;
+  size_t smem = idx_bytes + 2 * size_t(rps) * row_bytes;
   if (smem > 200 * 1024) {
     // rows too wide for two staged rows and the index table: one row at a time
     return inverse ? scatter(in, cols, out, cols, rows, rows, cols, map, nullptr, st, device)
@@ -337,17 +337,22 @@ cudaError_t permute_cols(const T* in, T* out, int64_t rows, int cols, const int3
   constexpr int kRegVecs = 8;
   const int vpr = cols / V;
   const bool reg_idx = (vpr + 255) / 256 <= kRegVecs;
+  // the register-index kernel keeps its table in stage 1 when it fits there
+  // (more blocks per SM for wide rows)
+  const int idx_in_stage = reg_idx && idx_bytes <= size_t(rps) * row_bytes ? 1 : 0;
+  if (idx_in_stage) smem = 2 * size_t(rps) * row_bytes;
   static bool attr_reg[64] = {false};
   cudaError_t e = reg_idx ? allow_smem(permute_rows_reg_kernel<T, kRegVecs>, smem, &attr_reg[device & 63])
                           : allow_smem(permute_rows_kernel<T>, smem, &attr[device & 63]);
   if (e != cudaSuccess) return e;
-  const int per_sm = static_cast<int>((220 * 1024) / (smem + 1024));
+  int per_sm = static_cast<int>((220 * 1024) / (smem + 1024));
+  if (reg_idx && per_sm > 3) per_sm = 3;  // its registers (76 per thread) fit three 256-thread blocks per SM
   const int64_t chunks = (rows + rps - 1) / rps;
   int64_t g = int64_t(sm_count(device)) * (per_sm < 1 ? 1 : (per_sm > 8 ? 8 : per_sm));
   if (g > chunks) g = chunks;
   if (reg_idx)
     permute_rows_reg_kernel<T, kRegVecs><<<static_cast<int>(g), 256, smem, st>>>(in, out, rows, cols, map, inverse,
-                                                                                 rps);
+                                                                                 rps, idx_in_stage);
   else
     permute_rows_kernel<T><<<static_cast<int>(g), 256, smem, st>>>(in, out, rows, cols, map, inverse, rps);
   return cudaGetLastError();
