@@ -133,8 +133,9 @@ poetx_status poetx_frame_export(const poetx_layer* layer, void* W0lin, void* str
  * (every power of Q is built from Q and S = Q^2).  POETX_FP32: fp32 FFMA;
  * POETX_BF16 with b = 256: one block per pair of SMs, every product on
  * tcgen05 tensor cores (cta_group::2) with bf16 operands and fp32
- * accumulation, G rounded once to bf16; POETX_BF16 with other b: a chain of
- * tcgen05 GEMMs with tf32 operands over the whole batch. */
+ * accumulation, S and H = 2Q + S kept in shared memory as bf16 operands,
+ * G = I + H + S + H S^T rounded once to bf16; POETX_BF16 with other b: a chain
+ * of tcgen05 GEMMs with tf32 operands over the whole batch. */
 poetx_status poetx_cnp_build(int32_t nblk, int32_t b, const float* q, int32_t dtype, void* G, void* ws,
                              size_t ws_bytes, void* stream);
 

@@ -20,6 +20,7 @@
 #include "quant.cuh"
 #include "adamw.cuh"
 #include "cnp2sm.cuh"
+#include "cnp2build.cuh"
 #include "bdg2sm.cuh"
 
 using namespace poetx;
@@ -611,6 +612,24 @@ cudaError_t launch_cnp_pair(const cnp2::PairSegs& sg_in, int nblk, bool backward
     PROFILED(ST_CNP_ELEM, st, cnp2::prep_kernel<false><<<pgrid, pblock, 0, st>>>(sg, region, nullptr));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  const uint32_t idesc_kk = (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(cnp2::BLK >> 3) << 17) |
+                            (static_cast<uint32_t>(cnp2::BLK >> 4) << 24);
+  if (!backward) {
+    // the build keeps S and H in shared memory (cnp2build.cuh)
+    static bool battr[64] = {false};
+    if (device >= 0 && device < 64 && !battr[device]) {
+      e = cudaFuncSetAttribute(cnp2b::cnp_build_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               cnp2b::SMEM_BYTES);
+      if (e != cudaSuccess) return e;
+      battr[device] = true;
+    }
+    cnp2b::Params bp;
+    bp.nblk = nblk;
+    bp.idesc = idesc_kk;
+    PROFILED(ST_CNP_GEMM, st,
+             cnp2b::cnp_build_pair_kernel<<<2 * pairs, cnp2b::NUM_THREADS, cnp2b::SMEM_BYTES, st>>>(mk, sg, bp));
+    return cudaGetLastError();
+  }
   cnp2::Params p;
   p.nblk = nblk;
   p.backward = backward ? 1 : 0;
