@@ -57,7 +57,7 @@ WORKLOAD = "block8b"
 # capture of that kernel and shape (dram__bytes_read.sum +
 # dram__bytes_write.sum); reset to None whenever the kernel changes until it
 # is captured again.
-W0_GEMM_TRAFFIC_BYTES = 1109613056 + 456707584
+W0_GEMM_TRAFFIC_BYTES = 948963840 + 455262208
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 NOMINAL_BF16_TFLOPS = 2250.0   # B200 dense bf16 tensor-core peak (datasheet, no sparsity)
 

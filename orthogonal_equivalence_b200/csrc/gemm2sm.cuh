@@ -30,11 +30,11 @@ constexpr int EPI_BOX = 32 * 128;
 constexpr int EPI_BYTES = 4 * 2 * EPI_BOX;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 1024 + 256;
 constexpr int NUM_THREADS = 192;
-constexpr int GROUP_M = 8;           // pair-tiles (256 rows each) per raster group
-
 struct Params {
   int M, N, K;
   int tiles_m, tiles_n;
+  int group;             // raster: panels per group along the grouped dimension
+  int group_n;           // 0: groups of M panels (A group held in L2, B streamed); 1: groups of N panels
   int b_mn;              // B operand MN-major (W~^T in the backward)
   uint32_t idesc;
   uint32_t b_lbo, b_kstep;
@@ -89,13 +89,19 @@ __device__ __forceinline__ void commit_pair(uint32_t bar) {
 }
 
 __device__ __forceinline__ void decode(const Params& p, int tile, int& mt, int& nt) {
-  const int group_span = GROUP_M * p.tiles_n;
-  const int g = tile / group_span;
-  const int first_m = g * GROUP_M;
-  const int gsize = min(p.tiles_m - first_m, GROUP_M);
-  const int r = tile - g * group_span;
-  mt = first_m + r % gsize;
-  nt = r / gsize;
+  // Tiles of one group share a set of `group` panels of the grouped dimension,
+  // which stay in L2 while the other dimension is swept (grouped dimension
+  // fastest, so the pairs of one wave read the same streamed panel together).
+  const int grouped = p.group_n ? p.tiles_n : p.tiles_m;
+  const int other = p.group_n ? p.tiles_m : p.tiles_n;
+  const int span = p.group * other;
+  const int g = tile / span;
+  const int first = g * p.group;
+  const int gsize = min(grouped - first, p.group);
+  const int r = tile - g * span;
+  const int a = first + r % gsize, b = r / gsize;
+  mt = p.group_n ? b : a;
+  nt = p.group_n ? a : b;
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
