@@ -109,53 +109,96 @@ __device__ __forceinline__ int chunk_type(int backward, int ph, int c) {
 }
 
 // ---------------------------------------------------------------- prep
-// Qb, and for the backward Gb and dq = 2 (dG[i][j] - dG[j][i]), of
-// the 32 x 32 tile pair (I, J), I <= J, of block blockIdx.y; grid (36, nblk),
-// block (32, 8).
+// Qb, and for the backward Gb and dq = 2 (dG[i][j] - dG[j][i]), of the
+// 64 x 64 tile pair (I, J), I <= J, of block blockIdx.y; grid (PREP_PAIRS,
+// nblk), PREP_THREADS threads.  Warp w handles rows w, w + 8, ... of a tile
+// and lane l its columns 2l and 2l + 1, so each warp store is one 128-byte
+// (bf16) or 256-byte (fp32) run, and a thread issues all of its loads
+// (16 triangle entries, 8 + 8 float2 of dG) before its first store.
+constexpr int PREP_T = 64;
+constexpr int PREP_TILES = BLK / PREP_T;
+constexpr int PREP_PAIRS = PREP_TILES * (PREP_TILES + 1) / 2;
+constexpr int PREP_THREADS = 256;
+constexpr int PREP_ROWS = PREP_T / (PREP_THREADS / 32);  // rows per warp
+
 template <bool BWD>
-__global__ void __launch_bounds__(256) prep_kernel(const __grid_constant__ PairSegs sg,
-                                                   __nv_bfloat16* __restrict__ Qb, __nv_bfloat16* __restrict__ Gb) {
-  __shared__ float tq[32][33];
-  __shared__ float g1[32][33];
-  __shared__ float g2[32][33];
+__global__ void __launch_bounds__(PREP_THREADS) prep_kernel(const __grid_constant__ PairSegs sg,
+                                                            __nv_bfloat16* __restrict__ Qb,
+                                                            __nv_bfloat16* __restrict__ Gb) {
+  __shared__ float tq[PREP_T][PREP_T + 1];                 // triangle entries of tile (I, J)
+  __shared__ float gs[BWD ? PREP_T : 1][PREP_T + 1];       // dG tile (J, I), read transposed
   const int t = blockIdx.y;
   int I = 0, x = blockIdx.x;
-  while (x >= 8 - I) {
-    x -= 8 - I;
+  while (x >= PREP_TILES - I) {
+    x -= PREP_TILES - I;
     ++I;
   }
   const int J = I + x;
   const int s = pair_seg_of(sg, t), lt = t - sg.start[s];
   const float* q = sg.q[s] + int64_t(lt) * TRI;
   __nv_bfloat16* Qt = Qb + size_t(t) * BLK * BLK;
-  const int tx = threadIdx.x, ty = threadIdx.y;
-  const float* dG = BWD ? sg.dG[s] + int64_t(lt) * BLK * BLK : nullptr;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c0 = 2 * lane;
+
+  // loads: the triangle's runs are not 8-byte aligned, so its entries come one
+  // float at a time (columns lane and lane + 32); dG rows come as float2
+  float v[PREP_ROWS][2];
 #pragma unroll
-  for (int r = ty; r < 32; r += 8) {
-    const int i = 32 * I + r, j = 32 * J + tx;
-    tq[r][tx] = j > i ? q[tri_index(i, j, BLK)] : 0.f;
+  for (int k = 0; k < PREP_ROWS; ++k) {
+    const int r = warp + 8 * k, i = PREP_T * I + r;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int j = PREP_T * J + lane + 32 * h;
+      v[k][h] = j > i ? q[tri_index(i, j, BLK)] : 0.f;
+    }
+  }
+  float2 g1[BWD ? PREP_ROWS : 1], g2[BWD ? PREP_ROWS : 1];
+  const float* dG = BWD ? sg.dG[s] + int64_t(lt) * BLK * BLK : nullptr;
+  if (BWD) {
+#pragma unroll
+    for (int k = 0; k < PREP_ROWS; ++k) {
+      const int r = warp + 8 * k;
+      g1[k] = *reinterpret_cast<const float2*>(dG + (PREP_T * I + r) * BLK + PREP_T * J + c0);
+      g2[k] = I < J ? *reinterpret_cast<const float2*>(dG + (PREP_T * J + r) * BLK + PREP_T * I + c0) : g1[k];
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < PREP_ROWS; ++k) {
+    const int r = warp + 8 * k;
+    tq[r][lane] = v[k][0];
+    tq[r][lane + 32] = v[k][1];
     if (BWD) {
-      g1[r][tx] = dG[i * BLK + j];
-      g2[r][tx] = dG[(32 * J + r) * BLK + 32 * I + tx];
+      gs[r][c0] = g2[k].x;
+      gs[r][c0 + 1] = g2[k].y;
     }
   }
   __syncthreads();
+
   float* dq = BWD ? static_cast<float*>(sg.out[s]) + int64_t(lt) * TRI : nullptr;
 #pragma unroll
-  for (int r = ty; r < 32; r += 8) {
-    const int i = 32 * I + r, j = 32 * J + tx;
-    // tile (I, J); for I < J also its mirror (J, I), Q[j][i] = -Q[i][j]
-    const float v = I < J ? tq[r][tx] : (j > i ? tq[r][tx] : (j < i ? -tq[tx][r] : 0.f));
-    Qt[i * BLK + j] = __float2bfloat16_rn(v);
-    if (I < J) Qt[(32 * J + r) * BLK + 32 * I + tx] = __float2bfloat16_rn(-tq[tx][r]);
+  for (int k = 0; k < PREP_ROWS; ++k) {
+    const int r = warp + 8 * k, i = PREP_T * I + r;
+    float a[2], m[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int c = c0 + e, j = PREP_T * J + c;
+      // tile (I, J); for I < J also its mirror (J, I), Q[j][i] = -Q[i][j]
+      a[e] = I < J ? tq[r][c] : (j > i ? tq[r][c] : (j < i ? -tq[c][r] : 0.f));
+      m[e] = -tq[c][r];
+    }
+    *reinterpret_cast<uint32_t*>(Qt + i * BLK + PREP_T * J + c0) = pack_bf16x2(a[0], a[1]);
+    if (I < J) *reinterpret_cast<uint32_t*>(Qt + (PREP_T * J + r) * BLK + PREP_T * I + c0) = pack_bf16x2(m[0], m[1]);
     if (BWD) {
       __nv_bfloat16* Gt = Gb + size_t(t) * BLK * BLK;
-      Gt[i * BLK + j] = __float2bfloat16_rn(g1[r][tx]);
-      if (I < J) Gt[(32 * J + r) * BLK + 32 * I + tx] = __float2bfloat16_rn(g2[r][tx]);
-      if (j > i) {
-        // dG[j][i]: g2 holds tile (J, I), the tile itself when I == J
-        const float gt = I < J ? g2[tx][r] : g1[tx][r];
-        dq[tri_index(i, j, BLK)] = 2.f * (g1[r][tx] - gt);
+      *reinterpret_cast<uint32_t*>(Gt + i * BLK + PREP_T * J + c0) = pack_bf16x2(g1[k].x, g1[k].y);
+      if (I < J)
+        *reinterpret_cast<uint32_t*>(Gt + (PREP_T * J + r) * BLK + PREP_T * I + c0) = pack_bf16x2(g2[k].x, g2[k].y);
+      const float gij[2] = {g1[k].x, g1[k].y};
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int c = c0 + e, j = PREP_T * J + c;
+        // dG[j][i]: gs holds tile (J, I), the tile itself when I == J
+        if (j > i) dq[tri_index(i, j, BLK)] = 2.f * (gij[e] - gs[c][r]);
       }
     }
   }

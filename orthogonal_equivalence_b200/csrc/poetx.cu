@@ -603,7 +603,7 @@ cudaError_t launch_cnp_pair(const cnp2::PairSegs& sg_in, int nblk, bool backward
   v.ld = cnp2::BLK;
   CUtensorMap mk, mm;
   if (!encode_map(&mk, v, cnp2::HALF) || !encode_map(&mm, v, cnp2::CH)) return cudaErrorInvalidValue;
-  const dim3 pgrid(36, nblk), pblock(32, 8);
+  const dim3 pgrid(cnp2::PREP_PAIRS, nblk), pblock(cnp2::PREP_THREADS);
   if (backward)
     PROFILED(ST_CNP_ELEM, st,
              cnp2::prep_kernel<true><<<pgrid, pblock, 0, st>>>(sg, region,
