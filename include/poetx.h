@@ -153,7 +153,7 @@ poetx_status poetx_layer_cnp_build(const poetx_layer* layer, void* ws, size_t ws
  * Scratch is a 24 MiB device array inside the library, held by every GPU
  * that loads it until the process exits.  It fits the build that runs:
  * POETX_BF16 with b = 256 (one block per pair of SMs) takes 128 KiB per block
- * plus 384 KiB per pair used, so nblk <= 47 on a 148-SM B200; the other
+ * (its bf16 Q), so nblk <= 191; the other
  * builds take Q, S and H in fp32, nblk*b*b <= ~2.09e6 elements (b = 512:
  * nblk <= 7; fp32 b = 64: nblk <= 511).  Larger requests return
  * POETX_E_WORKSPACE without queueing anything.  The

@@ -1,11 +1,11 @@
-// Cayley-Neumann build and backward for b = 256 blocks on CTA pairs (POET-X
-// write-up, section 3: G = (I+Q)(I+Q+Q^2+Q^3) from the packed skew Q, and
-// the gradient of the packed triangle).
+// Cayley-Neumann backward for b = 256 blocks on CTA pairs (POET-X write-up,
+// section 3: the gradient of the packed triangle of G = (I+Q)(I+Q+Q^2+Q^3)),
+// and the prep kernel it shares with the build (cnp2build.cuh).
 //
 // A grid-wide prep kernel first writes, for every block of the batch, Q in
 // bf16 (Qb) and, for the backward, dG in bf16 (Gb) and the part of dq that
-// needs no product, dq = 2 (dG[i][j] - dG[j][i]).  The fused kernel then takes one 256 x 256 block per pair
-// of SMs at a time: the leader CTA issues every product of the block back to
+// needs no product, dq = 2 (dG[i][j] - dG[j][i]).  The fused kernel then
+// takes one 256 x 256 block per pair of SMs at a time: the leader CTA issues every product of the block back to
 // back as tcgen05 MMAs with cta_group::2 (bf16 operands, fp32 accumulation),
 // each CTA keeping the accumulator rows of its half (rows 128*rank .. +127)
 // in its own TMEM.  Operands are read with TMA from Qb, Gb and a per-pair
@@ -14,20 +14,18 @@
 // is its rows and an MN-major tile its columns, so Q^T = -Q and dG^T, dS^T
 // need no copies.
 //
-// Build (S = Q^2 = -Q Q^T, H = 2Q + S, G = I + 2Q + 2S + H S^T):
-//   P1: acc0 = Q Q^T                          E1: S = -acc0, H = S + 2Q
-//   P2: acc1 = H S^T                          E2: G = I + 2Q + 2S + acc1
-// Backward (dS = 2dG + H^T dG + dG S, dA = 2dG + 2 dG S - dS Q - Q dS,
-// dq_k = dA[i][j] - dA[j][i] for k = k(i, j)):
+// With S = Q^2 = -Q Q^T and H = 2Q + S (G = I + 2Q + 2S + H S^T):
+// dS = 2dG + H^T dG + dG S, dA = 2dG + 2 dG S - dS Q - Q dS,
+// dq_k = dA[i][j] - dA[j][i] for k = k(i, j):
 //   P1: acc0 = Q Q^T                          E1: S = -acc0, H^T = S - 2Q
 //   P2: acc0 = H^T dG,  acc1 = dG S^T         E2: dS = 2dG + acc0 + acc1;
 //                                                 acc1 <- 2 acc1 (TMEM store)
 //   P3: acc1 += dS Q^T + Q^T dS               E3: acc1 (= dA - 2dG) -> smem
 //   F : dq += acc1[i][j] - acc1[j][i]  (the partner's rows through
 //       distributed shared memory; dq staged in shared memory by bulk copies)
-// The additive terms are added in fp32: S from the fp32 accumulator; I and
-// the 2dG of dq exactly (prep).  2Q in H and G and 2dG in dS, which only
-// feed bf16 operands or the bf16 G, use the bf16 copies the epilogue finds
+// The additive terms are added in fp32: S from the fp32 accumulator; the 2dG
+// of dq exactly (prep).  2Q in H^T and 2dG in dS, which only feed bf16
+// operands, use the bf16 copies the epilogue finds
 // in the staged operand tiles (the last four chunks of a phase always sit in
 // stages 0..3 when its epilogue runs).
 //
@@ -66,13 +64,13 @@ constexpr int DQ_HALF = static_cast<int>(TRI / 2);      // dq entries per CTA
 constexpr int DQ_BYTES = DQ_HALF * 4;                   // 65280, a multiple of 16
 constexpr int NUM_THREADS = 192;
 constexpr int SMEM_BYTES = REGION0 + DQ_BYTES + 256 + 1024;
-constexpr int SKINDS = 3;                // per-pair slot: S, H (H^T in the backward), dS
+constexpr int SKINDS = 3;                // per-pair slot: S, H^T, dS
 enum SlotKind : int { KS = 0, KH, KDS };
 constexpr size_t MAT_BYTES = size_t(BLK) * BLK * 2;
 
 // Operands of one K chunk: A and B are this CTA's rows (K-major) or, with a
 // "C" suffix, this CTA's columns (MN-major) of the named matrices.
-enum Chunk : int { C_QQ = 0, C_H_S, C_H_GC, C_G_S, C_DS_Q, C_QC_DSC };
+enum Chunk : int { C_QQ = 0, C_H_GC, C_G_S, C_DS_Q, C_QC_DSC };
 
 struct PairSegs {
   int n;
@@ -84,11 +82,10 @@ struct PairSegs {
 
 struct Params {
   int nblk;
-  int backward;
   uint32_t idesc_kk;       // A K-major, B K-major, M = N = 256
   uint32_t idesc_kmn;      // A K-major, B MN-major
   uint32_t idesc_mnmn;     // A MN-major, B MN-major
-  __nv_bfloat16* region;   // [Qb: nblk][Gb: nblk (backward)][slots: pairs x SKINDS], BLK x BLK each
+  __nv_bfloat16* region;   // [Qb: nblk][Gb: nblk][slots: pairs x SKINDS], BLK x BLK each
 };
 
 __device__ __forceinline__ int pair_seg_of(const PairSegs& sg, int blk) {
@@ -98,12 +95,9 @@ __device__ __forceinline__ int pair_seg_of(const PairSegs& sg, int blk) {
 }
 
 // Chunks of phase ph (1-based): count and type of chunk c.
-__device__ __forceinline__ int phase_chunks(int backward, int ph) {
-  return (backward && ph >= 2) ? 8 : 4;
-}
-__device__ __forceinline__ int chunk_type(int backward, int ph, int c) {
+__device__ __forceinline__ int phase_chunks(int ph) { return ph >= 2 ? 8 : 4; }
+__device__ __forceinline__ int chunk_type(int ph, int c) {
   if (ph == 1) return C_QQ;
-  if (!backward) return C_H_S;
   if (ph == 2) return c < 4 ? C_H_GC : C_G_S;
   return c < 4 ? C_DS_Q : C_QC_DSC;
 }
@@ -316,8 +310,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem_base = *tmem_holder;
 
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
-  const int nph = p.backward ? 3 : 2;
-  const int slot0 = (p.backward ? 2 : 1) * p.nblk + pair * SKINDS;  // matrix index of this pair's S
+  const int nph = 3;
+  const int slot0 = 2 * p.nblk + pair * SKINDS;  // matrix index of this pair's S
   auto matp = [&](int m) { return p.region + size_t(m) * BLK * BLK; };
   // shared-memory addresses of acc1's rows in both CTAs of the pair
   const uint32_t dA_cl0 = tc2::map_to_rank(smem_base, 0), dA_cl1 = tc2::map_to_rank(smem_base, 1);
@@ -345,10 +339,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     const int s = pair_seg_of(sg, blk);
     const int lt = blk - sg.start[s];
     const int mQ = blk, mG = p.nblk + blk;
-    float* dq_g = p.backward ? static_cast<float*>(sg.out[s]) + int64_t(lt) * TRI + int64_t(rank) * DQ_HALF
-                             : nullptr;
+    float* dq_g = static_cast<float*>(sg.out[s]) + int64_t(lt) * TRI + int64_t(rank) * DQ_HALF;
 
-    if (p.backward && threadIdx.x == 0 && !*s_abort) {
+    if (threadIdx.x == 0 && !*s_abort) {
       // this CTA's half of dq (2 (dG - dG^T) from the prep) into shared memory
       bulk_wait_read<0>();  // the previous block's store has read the staging buffer
       mbar_arrive_expect_tx(bar(DQ), DQ_BYTES);
@@ -356,7 +349,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     }
 
     for (int ph = 1; ph <= nph; ++ph) {
-      const int nch = phase_chunks(p.backward, ph);
+      const int nch = phase_chunks(ph);
       if (warp == 0) {
         if (lane == 0 && !*s_abort) {
           // ---------------- TMA producer
@@ -365,7 +358,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
               *s_abort = 1;
               break;
             }
-            const int type = chunk_type(p.backward, ph, c);
+            const int type = chunk_type(ph, c);
             const int k = (c & 3) * CH;
             const uint32_t full_leader = tc2::map_to_rank(bar(FULL + stage), 0);
             const uint32_t sa = smem_base + stage * STAGE_BYTES, sb = sa + TILE_BYTES;
@@ -380,7 +373,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             };
             switch (type) {
               case C_QQ: rows(sa, mQ); break;
-              case C_H_S: rows(sa, slot0 + KH); rows(sb, slot0 + KS); break;
               case C_H_GC: rows(sa, slot0 + KH); cols(sb, mG); break;
               case C_G_S: rows(sa, mG); rows(sb, slot0 + KS); break;
               case C_DS_Q: rows(sa, slot0 + KDS); rows(sb, mQ); break;
@@ -401,7 +393,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
               break;
             }
             tc_fence_after();
-            const int type = chunk_type(p.backward, ph, c);
+            const int type = chunk_type(ph, c);
             const uint32_t sa = smem_base + stage * STAGE_BYTES, sb = sa + TILE_BYTES;
             const bool a_mn = type == C_QC_DSC;
             const bool b_mn = type == C_H_GC || type == C_QC_DSC;
@@ -417,7 +409,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
               switch (type) {
                 case C_QQ:
                 case C_H_GC: tc2::mma_pair(acc0, da, db, id, fresh); break;
-                case C_H_S:
                 case C_G_S: tc2::mma_pair(acc1, da, db, id, fresh); break;
                 default: tc2::mma_pair(acc1, da, db, id, 1u); break;  // P3 adds to 2 dG S^T
               }
@@ -439,12 +430,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           float v0[32], v1[32], w[32];
           // 64 columns per step: the TMEM loads of a step share one round trip
           for (int c0 = 0; c0 < BLK; c0 += 64) {
-            const uint32_t tileA = smem_base + (c0 >> 6) * STAGE_BYTES, tileB = tileA + TILE_BYTES;
+            const uint32_t tileA = smem_base + (c0 >> 6) * STAGE_BYTES;
             if (ph == 1) {
-              // S = -acc0;  H = S + 2Q (build) or H^T = S - 2Q (backward); Q from P1's A tiles
+              // S = -acc0;  H^T = S - 2Q; Q from P1's A tiles
               float a1[32];
               tmem_ld_32cols_x2(t0 + c0, t0 + c0 + 32, v0, a1);
-              const float sgn = p.backward ? -2.f : 2.f;
 #pragma unroll
               for (int h = 0; h < 2; ++h) {
                 const int cc = c0 + 32 * h;
@@ -453,25 +443,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
                   a[e] = -a[e];
-                  v1[e] = a[e] + sgn * w[e];
+                  v1[e] = a[e] - 2.f * w[e];
                 }
                 store_bf16x32(matp(slot0 + KS) + row * BLK + cc, a);
                 store_bf16x32(matp(slot0 + KH) + row * BLK + cc, v1);
-              }
-            } else if (!p.backward) {
-              // G = I + 2Q + 2S + acc1, 2Q = H - S from P2's A (H) and B (S) tiles, S = -acc0
-#pragma unroll 1
-              for (int h = 0; h < 2; ++h) {
-                const int cc = c0 + 32 * h;
-                tmem_ld_32cols_x2(t0 + cc, t0 + BLK + cc, v0, v1);
-                tile_row_bf16x32(tileA, lrow, cc, w);
-                float sb[32];
-                tile_row_bf16x32(tileB, lrow, cc, sb);
-#pragma unroll
-                for (int e = 0; e < 32; ++e)
-                  v1[e] = ((cc + e == row ? 1.f : 0.f) + (w[e] - sb[e])) + (-2.f * v0[e]) + v1[e];
-                __nv_bfloat16* G = static_cast<__nv_bfloat16*>(sg.out[s]) + int64_t(lt) * BLK * BLK;
-                store_bf16x32(G + row * BLK + cc, v1);
               }
             } else if (ph == 2) {
               // dS = 2dG + acc0 + acc1 (a bf16 operand; dG from P2's A tiles); acc1 <- 2 acc1
@@ -505,7 +480,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       phase_barrier();
     }
 
-    if (p.backward) {
+    {
       // ---------------- F: this CTA's half of dq, k in [rank * DQ_HALF, +DQ_HALF)
       bool ok = !*s_abort && mbar_wait(bar(DQ), dq_phase, DERR_GEMM_WAIT);
       dq_phase ^= 1u;

@@ -557,7 +557,8 @@ Segs two_segs(const float* q0, int n0, void* G0, const float* q1, int n1, void* 
 // Up to two segments write G straight from the GEMM epilogue; more go
 // through a contiguous scratch copy (`gall`, nblk*b*b elements of dtype).
 // ---- fused CNP on CTA pairs (b = 256, bf16 layers): one kernel per batch,
-// every product of a block on tcgen05 with the operands in an L2-resident
+// every product of a block on tcgen05; the build keeps its operands in shared
+// memory (cnp2build.cuh), the backward passes them through an L2-resident
 // per-pair slot (cnp2sm.cuh).
 bool use_pair_cnp(int32_t b, int32_t dtype) { return b == cnp2::BLK && dtype == POETX_BF16; }
 
@@ -566,10 +567,13 @@ int cnp_pair_count(int nblk, int device) {
   return nblk < pairs ? nblk : pairs;
 }
 
+// bf16 operand region: the build's Q (nblk matrices); the backward's Q, dG
+// and the per-pair slots (plus an fp32 dq scratch when it accumulates)
 size_t cnp_pair_bytes(int nblk, bool backward, bool accumulate, int device) {
+  if (!backward) return al(size_t(nblk) * cnp2::MAT_BYTES);
   const int pairs = cnp_pair_count(nblk, device);
-  return al((size_t(nblk) * (backward ? 2 : 1) + size_t(pairs) * cnp2::SKINDS) * cnp2::MAT_BYTES) +
-         (backward && accumulate ? al(sizeof(float) * size_t(nblk) * cnp2::TRI) : 0);
+  return al((size_t(nblk) * 2 + size_t(pairs) * cnp2::SKINDS) * cnp2::MAT_BYTES) +
+         (accumulate ? al(sizeof(float) * size_t(nblk) * cnp2::TRI) : 0);
 }
 
 // Prep (bf16 Q, and for the backward bf16 dG and dq = 2 (dG - dG^T)) and the
@@ -587,7 +591,7 @@ cudaError_t launch_cnp_pair(const cnp2::PairSegs& sg_in, int nblk, bool backward
   }
   const int pairs = cnp_pair_count(nblk, device);
   if (pairs <= 0) return cudaSuccess;
-  const int nmat = nblk * (backward ? 2 : 1) + pairs * cnp2::SKINDS;
+  const int nmat = backward ? 2 * nblk + pairs * cnp2::SKINDS : nblk;
   __nv_bfloat16* region = ws.take<__nv_bfloat16>(size_t(nmat) * cnp2::MAT_BYTES);
   cnp2::PairSegs sg = sg_in;
   float* dq_tmp = nullptr;
@@ -632,7 +636,6 @@ cudaError_t launch_cnp_pair(const cnp2::PairSegs& sg_in, int nblk, bool backward
   }
   cnp2::Params p;
   p.nblk = nblk;
-  p.backward = backward ? 1 : 0;
   // D fp32, A and B bf16, N = 256 (bits 17-22: N >> 3), M = 256 (bits 24-28: M >> 4);
   // bit 15: A MN-major, bit 16: B MN-major
   p.idesc_kk = (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(cnp2::BLK >> 3) << 17) |
