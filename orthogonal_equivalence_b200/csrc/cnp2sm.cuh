@@ -62,8 +62,24 @@ constexpr int REGION0 = ((RING_BYTES > DA_SMEM ? RING_BYTES : DA_SMEM) + 1023) &
 constexpr int64_t TRI = int64_t(BLK) * (BLK - 1) / 2;
 constexpr int DQ_HALF = static_cast<int>(TRI / 2);      // dq entries per CTA
 constexpr int DQ_BYTES = DQ_HALF * 4;                   // 65280, a multiple of 16
+// The fold splits the triangle into eight bands of 32 rows; band I holds the
+// entries of rows 32I .. 32I+31 (7664 - 1024 I of them, a contiguous run of
+// dq).  CTA 0 folds bands 0, 3, 4, 7 and CTA 1 bands 1, 2, 5, 6: 16320
+// entries and 18 tiles of 32 x 32 each.
+constexpr int BANDS = BLK / 32;
+__host__ __device__ constexpr int band_of(int rank, int b) {
+  return rank == 0 ? (b == 0 ? 0 : b == 1 ? 3 : b == 2 ? 4 : 7) : (b == 0 ? 1 : b == 1 ? 2 : b == 2 ? 5 : 6);
+}
+__host__ __device__ constexpr int band_start(int I) { return I * (2 * BLK - 1 - 32 * I) * 16; }  // tri_index(32I, 32I+1)
+__host__ __device__ constexpr int band_size(int I) { return band_start(I + 1) - band_start(I); }
+static_assert(band_start(BANDS) == TRI, "bands cover the triangle");
+static_assert(band_size(0) + band_size(3) + band_size(4) + band_size(7) == DQ_HALF &&
+                  band_size(1) + band_size(2) + band_size(5) + band_size(6) == DQ_HALF,
+              "each CTA folds half of dq");
 constexpr int NUM_THREADS = 192;
-constexpr int SMEM_BYTES = REGION0 + DQ_BYTES + 256 + 1024;
+constexpr int TT_LD = 33;                // padded row of a warp's 32 x 32 transpose tile
+constexpr int TT_BYTES = (NUM_THREADS / 32) * 32 * TT_LD * 4;
+constexpr int SMEM_BYTES = REGION0 + DQ_BYTES + 256 + TT_BYTES + 1024;
 constexpr int SKINDS = 3;                // per-pair slot: S, H^T, dS
 enum SlotKind : int { KS = 0, KH, KDS };
 constexpr size_t MAT_BYTES = size_t(BLK) * BLK * 2;
@@ -274,11 +290,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* dAs = reinterpret_cast<float*>(smem);                // acc1 rows after P3 (over the ring)
-  float* dqs = reinterpret_cast<float*>(smem + REGION0);      // this CTA's half of the block's dq
+  float* dqs = reinterpret_cast<float*>(smem + REGION0);      // this CTA's four bands of the block's dq
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + REGION0 + DQ_BYTES);
   // bars: full[STAGES] (leader), empty[STAGES], acc, dq
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 2);
   volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  float* tt = reinterpret_cast<float*>(smem + REGION0 + DQ_BYTES + 256) + (threadIdx.x >> 5) * 32 * TT_LD;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -339,13 +356,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     const int s = pair_seg_of(sg, blk);
     const int lt = blk - sg.start[s];
     const int mQ = blk, mG = p.nblk + blk;
-    float* dq_g = static_cast<float*>(sg.out[s]) + int64_t(lt) * TRI + int64_t(rank) * DQ_HALF;
+    float* dq_g = static_cast<float*>(sg.out[s]) + int64_t(lt) * TRI;
 
     if (threadIdx.x == 0 && !*s_abort) {
       // this CTA's half of dq (2 (dG - dG^T) from the prep) into shared memory
       bulk_wait_read<0>();  // the previous block's store has read the staging buffer
       mbar_arrive_expect_tx(bar(DQ), DQ_BYTES);
-      bulk_load(smem_u32(dqs), dq_g, DQ_BYTES, bar(DQ));
+      for (int b = 0, off = 0; b < 4; off += band_size(band_of(rank, b)), ++b)
+        bulk_load(smem_u32(dqs + off), dq_g + band_start(band_of(rank, b)), band_size(band_of(rank, b)) * 4,
+                  bar(DQ));
     }
 
     for (int ph = 1; ph <= nph; ++ph) {
@@ -481,55 +500,56 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     }
 
     {
-      // ---------------- F: this CTA's half of dq, k in [rank * DQ_HALF, +DQ_HALF)
+      // ---------------- F: this CTA's four bands of dq
       bool ok = !*s_abort && mbar_wait(bar(DQ), dq_phase, DERR_GEMM_WAIT);
       dq_phase ^= 1u;
       if (!ok) *s_abort = 1;
       __syncwarp();
       if (!*s_abort) {
-        // element e = tid + 192 m of this CTA's range, k = k0 + e; the row of
-        // k advances monotonically with m.  Loads are issued eight elements
-        // (sixteen loads) at a time.
-        const int k0 = int(rank) * DQ_HALF;
-        const int tid = threadIdx.x;
-        int lo = 0, hi = BLK - 2;  // the row i with start(i) <= k0 + tid < start(i + 1)
-        while (lo < hi) {
-          const int mid = (lo + hi + 1) >> 1;
-          if (tri_index(mid, mid + 1, BLK) <= k0 + tid) lo = mid;
-          else hi = mid - 1;
-        }
-        int i = lo;
-        int ks = static_cast<int>(tri_index(i, i + 1, BLK)), ke = ks + (BLK - 1 - i);
-        for (int m0 = 0; m0 * NUM_THREADS < DQ_HALF; m0 += 8) {
-          float a[8], b[8];
-          int idx[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const int e = tid + NUM_THREADS * (m0 + u);
-            idx[u] = e < DQ_HALF ? e : -1;
-            if (idx[u] < 0) continue;
-            const int k = k0 + e;
-            while (k >= ke) {
-              ++i;
-              ks = ke;
-              ke = ks + (BLK - 1 - i);
-            }
-            const int j = i + 1 + (k - ks);
-            const uint32_t aij = (i < HALF ? dA_cl0 : dA_cl1) + uint32_t((i & (HALF - 1)) * DA_LD + j) * 4u;
-            const uint32_t aji = (j < HALF ? dA_cl0 : dA_cl1) + uint32_t((j & (HALF - 1)) * DA_LD + i) * 4u;
-            a[u] = ld_cluster_f32(aij);
-            b[u] = ld_cluster_f32(aji);
+        // Warp w folds tiles w, w + 6, w + 12 of this CTA's 18 (band I, tile
+        // column J >= I).  Lane l holds column j = 32J + l.  Every load reads
+        // one row with the lanes on consecutive columns (one request per warp,
+        // local or from the partner CTA): a[r] = acc1[32I + r][j] and u[r] =
+        // acc1[32J + r][32I + l]; u is transposed through the warp's own
+        // padded tile, so lane l gets acc1[j][32I + r].  All 64 loads are
+        // issued before use.
+        for (int tile = warp; tile < 18; tile += NUM_THREADS / 32) {
+          int b = 0, rest = tile, off = 0;
+          while (rest >= BANDS - band_of(rank, b)) {
+            rest -= BANDS - band_of(rank, b);
+            off += band_size(band_of(rank, b));
+            ++b;
           }
+          const int I = band_of(rank, b), J = I + rest;
+          const int i0 = 32 * I, j = 32 * J + lane;
+          const int j0 = 32 * J;
+          const uint32_t rowI = (i0 < HALF ? dA_cl0 : dA_cl1) + uint32_t((i0 & (HALF - 1)) * DA_LD + j) * 4u;
+          const uint32_t rowJ = (j0 < HALF ? dA_cl0 : dA_cl1) + uint32_t((j0 & (HALF - 1)) * DA_LD + i0 + lane) * 4u;
+          float a[32], t[32];
 #pragma unroll
-          for (int u = 0; u < 8; ++u)
-            if (idx[u] >= 0) dqs[idx[u]] += a[u] - b[u];
+          for (int r = 0; r < 32; ++r) a[r] = ld_cluster_f32(rowI + uint32_t(r * DA_LD) * 4u);
+#pragma unroll
+          for (int r = 0; r < 32; ++r) t[r] = ld_cluster_f32(rowJ + uint32_t(r * DA_LD) * 4u);
+#pragma unroll
+          for (int r = 0; r < 32; ++r) tt[r * TT_LD + lane] = t[r];
+          __syncwarp();
+#pragma unroll
+          for (int r = 0; r < 32; ++r) t[r] = tt[lane * TT_LD + r];
+          __syncwarp();
+          const int base = off - band_start(I);  // dqs index of entry k is base + k
+#pragma unroll
+          for (int r = 0; r < 32; ++r) {
+            const int i = i0 + r;
+            if (j > i) dqs[base + static_cast<int>(tri_index(i, j, BLK))] += a[r] - t[r];
+          }
         }
       }
       fence_proxy_async_all();
       __syncthreads();
       tc2::cluster_sync();  // both CTAs are done reading each other's rows; staging complete
       if (threadIdx.x == 0 && !*s_abort) {
-        bulk_store(dq_g, smem_u32(dqs), DQ_BYTES);
+        for (int b = 0, off = 0; b < 4; off += band_size(band_of(rank, b)), ++b)
+          bulk_store(dq_g + band_start(band_of(rank, b)), smem_u32(dqs + off), band_size(band_of(rank, b)) * 4);
         bulk_commit();
       }
     }
