@@ -9,8 +9,9 @@
 // back as tcgen05 MMAs with cta_group::2 (bf16 operands, fp32 accumulation),
 // each CTA keeping the accumulator rows of its half (rows 128*rank .. +127)
 // in its own TMEM.  Operands are read with TMA from Qb, Gb and a per-pair
-// slot (S, H, dS, written by the previous epilogue; one slot per pair,
-// reused block after block, so it stays in L2).  A K-major tile of a matrix
+// slot (S, H^T, dS, written by the previous epilogue with TMA stores from
+// swizzled 32-row boxes; one slot per pair, reused block after block, so it
+// stays in L2).  A K-major tile of a matrix
 // is its rows and an MN-major tile its columns, so Q^T = -Q and dG^T, dS^T
 // need no copies.
 //
@@ -55,6 +56,7 @@ constexpr int UMMA_K = 16;
 constexpr int TILE_BYTES = HALF * 128;   // 128 rows x 64 bf16, or 64 rows x 2 x 64 (MN-major)
 constexpr int STAGE_BYTES = 2 * TILE_BYTES;
 constexpr int STAGES = 4;
+constexpr int EPI_BOX = 32 * 128;        // 32 rows x 64 bf16: one TMA store of an epilogue warp
 constexpr int RING_BYTES = STAGES * STAGE_BYTES;
 constexpr int DA_LD = BLK + 1;           // padded fp32 row of acc1 in shared memory
 constexpr int DA_SMEM = HALF * DA_LD * 4;
@@ -101,8 +103,8 @@ struct Params {
   uint32_t idesc_kk;       // A K-major, B K-major, M = N = 256
   uint32_t idesc_kmn;      // A K-major, B MN-major
   uint32_t idesc_mnmn;     // A MN-major, B MN-major
-  __nv_bfloat16* region;   // [Qb: nblk][Gb: nblk][slots: pairs x SKINDS], BLK x BLK each
 };
+// The operand region the tensor maps cover: [Qb: nblk][Gb: nblk][slots: pairs x SKINDS], BLK x BLK bf16 each.
 
 __device__ __forceinline__ int pair_seg_of(const PairSegs& sg, int blk) {
   int s = 0;
@@ -271,6 +273,20 @@ __device__ __forceinline__ void tile_row_bf16x32(uint32_t tile, int r, int c0, f
     }
   }
 }
+// 32 values of row r (0..31), columns 32h .. 32h+31, of a 32-row x 64-column
+// bf16 box with 128-byte swizzle (16-byte chunk u of a row at u ^ (r % 8)),
+// the layout a TMA store of that box reads.
+__device__ __forceinline__ void box_row_bf16x32(uint32_t box, int r, int h, const float* v) {
+  const uint32_t rowp = box + r * 128;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const uint32_t w0 = pack_bf16x2(v[8 * u], v[8 * u + 1]), w1 = pack_bf16x2(v[8 * u + 2], v[8 * u + 3]);
+    const uint32_t w2 = pack_bf16x2(v[8 * u + 4], v[8 * u + 5]), w3 = pack_bf16x2(v[8 * u + 6], v[8 * u + 7]);
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(rowp + (((4 * h + u) ^ (r & 7)) << 4)), "r"(w0),
+                 "r"(w1), "r"(w2), "r"(w3)
+                 : "memory");
+  }
+}
 __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* p, const float* v) {
   uint4* d = reinterpret_cast<uint4*>(p);
 #pragma unroll
@@ -286,7 +302,7 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* p, const float* v) 
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     cnp_pair_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmMN,
-                    const __grid_constant__ PairSegs sg, const Params p) {
+                    const __grid_constant__ CUtensorMap tmS, const __grid_constant__ PairSegs sg, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* dAs = reinterpret_cast<float*>(smem);                // acc1 rows after P3 (over the ring)
@@ -329,7 +345,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const int nph = 3;
   const int slot0 = 2 * p.nblk + pair * SKINDS;  // matrix index of this pair's S
-  auto matp = [&](int m) { return p.region + size_t(m) * BLK * BLK; };
   // shared-memory addresses of acc1's rows in both CTAs of the pair
   const uint32_t dA_cl0 = tc2::map_to_rank(smem_base, 0), dA_cl1 = tc2::map_to_rank(smem_base, 1);
 
@@ -350,7 +365,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 
   const int quarter = warp & 3;
   const int lrow = quarter * 32 + lane;           // this thread's row of the CTA's half in the epilogues
-  const int row = int(rank) * HALF + lrow;        // and of the block
 
   for (int blk = pair; blk < p.nblk; blk += npairs) {
     const int s = pair_seg_of(sg, blk);
@@ -446,10 +460,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         } else {
           tc_fence_after();
           const uint32_t t0 = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+          // E1 and E2 stage their bf16 rows in 32-row x 64-column boxes and
+          // write them with TMA stores: the B tile of ring stage `quarter` is
+          // free then (P1 loads only A tiles; P2's last B tiles, S, are read)
+          const uint32_t stg = smem_base + quarter * STAGE_BYTES + TILE_BYTES;
+          const int grow = int(rank) * HALF + quarter * 32;  // this warp's first row of a slot matrix
           float v0[32], v1[32], w[32];
           // 64 columns per step: the TMEM loads of a step share one round trip
           for (int c0 = 0; c0 < BLK; c0 += 64) {
             const uint32_t tileA = smem_base + (c0 >> 6) * STAGE_BYTES;
+            if (ph <= 2) {
+              if (lane == 0) bulk_wait_read<1>();  // the boxes of two steps ago have been read
+              __syncwarp();
+            }
             if (ph == 1) {
               // S = -acc0;  H^T = S - 2Q; Q from P1's A tiles
               float a1[32];
@@ -464,8 +487,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                   a[e] = -a[e];
                   v1[e] = a[e] - 2.f * w[e];
                 }
-                store_bf16x32(matp(slot0 + KS) + row * BLK + cc, a);
-                store_bf16x32(matp(slot0 + KH) + row * BLK + cc, v1);
+                const uint32_t bS = stg + ((c0 >> 6) & 1) * 2 * EPI_BOX;
+                box_row_bf16x32(bS, lane, h, a);
+                box_row_bf16x32(bS + EPI_BOX, lane, h, v1);
+              }
+              fence_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                const uint32_t bS = stg + ((c0 >> 6) & 1) * 2 * EPI_BOX;
+                tma_store_2d(&tmS, bS, c0, (slot0 + KS) * BLK + grow);
+                tma_store_2d(&tmS, bS + EPI_BOX, c0, (slot0 + KH) * BLK + grow);
+                bulk_commit();
               }
             } else if (ph == 2) {
               // dS = 2dG + acc0 + acc1 (a bf16 operand; dG from P2's A tiles); acc1 <- 2 acc1
@@ -479,8 +511,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                   v0[e] = (2.f * w[e] + v0[e]) + v1[e];
                   v1[e] = 2.f * v1[e];
                 }
-                store_bf16x32(matp(slot0 + KDS) + row * BLK + cc, v0);
+                box_row_bf16x32(stg + ((c0 >> 6) & 1) * EPI_BOX, lane, h, v0);
                 tmem_st_32cols(t0 + BLK + cc, v1);
+              }
+              fence_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_2d(&tmS, stg + ((c0 >> 6) & 1) * EPI_BOX, c0, (slot0 + KDS) * BLK + grow);
+                bulk_commit();
               }
             } else {
               // acc1 = dA - 2dG for the fold (padded rows: conflict-free transposed reads)
@@ -493,6 +531,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
               }
             }
           }
+          // the slot rows are complete in global memory before the phase barrier
+          if (lane == 0) bulk_wait_all();
+          __syncwarp();
         }
       }
       acc_phase ^= 1u;

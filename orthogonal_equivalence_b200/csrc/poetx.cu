@@ -605,8 +605,9 @@ cudaError_t launch_cnp_pair(const cnp2::PairSegs& sg_in, int nblk, bool backward
   v.rows = int64_t(nmat) * cnp2::BLK;
   v.cols = cnp2::BLK;
   v.ld = cnp2::BLK;
-  CUtensorMap mk, mm;
-  if (!encode_map(&mk, v, cnp2::HALF) || !encode_map(&mm, v, cnp2::CH)) return cudaErrorInvalidValue;
+  CUtensorMap mk, mm, ms;
+  if (!encode_map(&mk, v, cnp2::HALF) || !encode_map(&mm, v, cnp2::CH) || !encode_map(&ms, v, 32))
+    return cudaErrorInvalidValue;
   const dim3 pgrid(cnp2::PREP_PAIRS, nblk), pblock(cnp2::PREP_THREADS);
   if (backward)
     PROFILED(ST_CNP_ELEM, st,
@@ -642,9 +643,8 @@ cudaError_t launch_cnp_pair(const cnp2::PairSegs& sg_in, int nblk, bool backward
                (static_cast<uint32_t>(cnp2::BLK >> 4) << 24);
   p.idesc_kmn = p.idesc_kk | (1u << 16);
   p.idesc_mnmn = p.idesc_kk | (1u << 15) | (1u << 16);
-  p.region = region;
   PROFILED(ST_CNP_GEMM, st,
-           cnp2::cnp_pair_kernel<<<2 * pairs, cnp2::NUM_THREADS, cnp2::SMEM_BYTES, st>>>(mk, mm, sg, p));
+           cnp2::cnp_pair_kernel<<<2 * pairs, cnp2::NUM_THREADS, cnp2::SMEM_BYTES, st>>>(mk, mm, ms, sg, p));
   e = cudaGetLastError();
   if (e != cudaSuccess || !dq_tmp) return e;
   for (int i = 0; i < sg.n; ++i) {
