@@ -44,6 +44,12 @@ struct Params {
   uint32_t idesc;                 // A K-major, B K-major, M = N = 256
 };
 
+// One tensor map per segment over its G ([blocks * 256][256] bf16, boxes of
+// 32 rows x 64 columns, 128-byte swizzle): E2 writes G with TMA stores.
+struct GMaps {
+  CUtensorMap m[kMaxSegs];
+};
+
 // 32 bf16 of row r, columns c0 .. c0+31 (c0 % 32 == 0), into the 128-byte
 // swizzled K-major tiles of a 128 x 256 matrix (tile c0 / 64; 16-byte chunk u
 // of a row sits at chunk u ^ (r % 8)).
@@ -62,7 +68,7 @@ __device__ __forceinline__ void tile_row_store_bf16x32(uint32_t mat, int r, int 
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     cnp_build_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ cnp2::PairSegs sg,
-                          const Params p) {
+                          const __grid_constant__ GMaps gm, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 3 * MAT_BYTES);
@@ -207,7 +213,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         break;
       }
       tc_fence_after();
-      __nv_bfloat16* G = static_cast<__nv_bfloat16*>(sg.out[s]) + int64_t(lt) * BLK * BLK + int64_t(row) * BLK;
+      // G replaces S in this warp's 32 rows of each tile (S and H of a row are
+      // read before its G is written), and each 32-row x 64-column box goes
+      // out with one TMA store
       for (int c0 = 0; c0 < BLK; c0 += 64) {
         float a[32], b[32], hs[32], sv[32];
         tmem_ld_32cols_x2(t0 + BLK + c0, t0 + BLK + c0 + 32, a, b);
@@ -219,13 +227,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           cnp2::tile_row_bf16x32(sS + (cc >> 6) * TILE_BYTES, lrow, cc, sv);
 #pragma unroll
           for (int e = 0; e < 32; ++e) v[e] = ((cc + e == row ? 1.f : 0.f) + (hs[e] + sv[e])) + v[e];
-          cnp2::store_bf16x32(G + cc, v);
+          tile_row_store_bf16x32(sS, lrow, cc, v);
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&gm.m[s], sS + (c0 >> 6) * TILE_BYTES + quarter * 32 * 128, c0, lt * BLK + row - lane);
+          bulk_commit();
         }
       }
+      // the next block's E1 writes S again: the stores have read it
+      if (lane == 0) bulk_wait_read<0>();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) tc2::remote_arrive(a1empty_leader);
     }
+    if (lane == 0) bulk_wait_all();  // G is in global memory before the block leaves
   }
 
   if (*s_abort && threadIdx.x == 0) {

@@ -631,8 +631,18 @@ cudaError_t launch_cnp_pair(const cnp2::PairSegs& sg_in, int nblk, bool backward
     cnp2b::Params bp;
     bp.nblk = nblk;
     bp.idesc = idesc_kk;
+    cnp2b::GMaps gm;
+    for (int i = 0; i < sg.n; ++i) {
+      Operand2D g;
+      g.ptr = sg.out[i];
+      g.et = ET_BF16;
+      g.rows = int64_t(sg.start[i + 1] - sg.start[i]) * cnp2::BLK;
+      g.cols = cnp2::BLK;
+      g.ld = cnp2::BLK;
+      if (g.rows > 0 && !encode_map(&gm.m[i], g, 32)) return cudaErrorInvalidValue;
+    }
     PROFILED(ST_CNP_GEMM, st,
-             cnp2b::cnp_build_pair_kernel<<<2 * pairs, cnp2b::NUM_THREADS, cnp2b::SMEM_BYTES, st>>>(mk, sg, bp));
+             cnp2b::cnp_build_pair_kernel<<<2 * pairs, cnp2b::NUM_THREADS, cnp2b::SMEM_BYTES, st>>>(mk, sg, gm, bp));
     return cudaGetLastError();
   }
   cnp2::Params p;
