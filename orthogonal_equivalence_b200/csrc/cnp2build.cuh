@@ -9,7 +9,9 @@
 //   E1: S = -acc0, H = S + 2Q, both written as bf16 operand tiles into this
 //       CTA's shared memory (the 128-byte swizzled K-major layout TMA uses)
 //   P2: acc1 = H S^T   A = this CTA's rows of H, B = its rows of S
-//   E2: G = I + H + S + acc1, rounded once to bf16
+//   E2: G = I + H + S + acc1, rounded once to bf16, written over this
+//       warp's rows of S and sent to global memory by TMA stores of
+//       32-row x 64-column boxes
 // so no operand leaves the SM between the phases (the kernel used for the
 // backward stages S, H through L2).  Q of the next block is loaded as soon as
 // E1 has read this block's Q, and P1 of the next block runs during E2 of this
