@@ -148,7 +148,7 @@ poetx_status poetx_layer_cnp_build(const poetx_layer* layer, void* ws, size_t ws
 /* poetx_cnp_build without a caller workspace, for callers that cannot
  * allocate device memory (for example a host program with no device
  * allocator of its own, or a process that fixes its memory budget at
- * start-up).  The paper has no counterpart: this is a deployment variant of
+ * start-up).  The write-up has no counterpart: this is a deployment variant of
  * poetx_cnp_build with the same arguments (minus ws) and the same result.
  * Scratch is a 24 MiB device array inside the library, held by every GPU
  * that loads it until the process exits.  It fits the build that runs:

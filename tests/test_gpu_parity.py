@@ -480,6 +480,29 @@ def test_dG_backward_and_batched_cnp_backward(case):
     assert np.array_equal(bits(acc), bits(2 * dG))
 
 
+def test_batched_build_of_the_most_layers_one_call_takes():
+    # 16 linears = 32 segments, the most one batched call takes: every
+    # segment's G (its own output buffer) equals the per-layer build, and the
+    # oracle on a few of them; one more linear is refused before any launch
+    shapes = [(256, 256), (512, 256), (256, 512), (512, 512)] * 4
+    inps = [_inputs("block8b", m, n, None, 8, layer=k) for k, (m, n) in enumerate(shapes)]
+    Ls = [make_layer(i) for i in inps]
+    ref = [(L.GR.clone(), L.GP.clone()) for L in Ls]
+    for L in Ls:
+        L.GR.fill_(float("nan"))
+        L.GP.fill_(float("nan"))
+    px.LayerGroup(Ls).build()
+    torch.cuda.synchronize()
+    for k, (L, inp, (gr, gp)) in enumerate(zip(Ls, inps, ref)):
+        assert np.array_equal(bits(L.GR), bits(gr)) and np.array_equal(bits(L.GP), bits(gp)), f"layer {k}"
+        if k in (0, 7, 15):
+            check(host64(L.GR), oracle.cnp_blocks(inp.qR, inp.b), inp.dtype, f"GR of layer {k}")
+            check(host64(L.GP), oracle.cnp_blocks(inp.qP, inp.b), inp.dtype, f"GP of layer {k}")
+    extra = make_layer(_inputs("block8b", 256, 256, None, 8, layer=16))
+    with pytest.raises(px.PoetxError):
+        px.LayerGroup(Ls + [extra]).build()
+
+
 def test_layer_group_batched_cnp_backward():
     """Several linears: backward_dG of each into one flat dG buffer, then one
     batched CNP backward into the flat dq, equals each layer's own dq."""
