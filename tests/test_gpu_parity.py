@@ -99,6 +99,32 @@ def test_layer_forward_backward_parity(case):
     check(host64(dqP), dqPo, inp.dtype, "dqP")
 
 
+def _skew_from_packed(p, b):
+    # packed upper triangles [nblk][b(b-1)/2] (row-major over i < j) -> [nblk][b][b], lower part zero
+    out = np.zeros((p.shape[0], b, b))
+    iu = np.triu_indices(b, 1)
+    out[:, iu[0], iu[1]] = p
+    return out
+
+
+def _tilewise(a, o, what, tile=32, bar=3e-2):
+    # relative Frobenius error of every 32 x 32 tile of every block (tiles whose
+    # reference is all zero, i.e. the empty lower tiles of a packed triangle,
+    # must be zero too), so that one wrong tile cannot hide in the whole-block norm
+    nblk, b, _ = o.shape
+    t = min(tile, b)
+    for k in range(nblk):
+        for I in range(0, b, t):
+            for J in range(0, b, t):
+                at, ot = a[k, I:I + t, J:J + t], o[k, I:I + t, J:J + t]
+                no = np.linalg.norm(ot)
+                if no == 0:
+                    assert np.all(at == 0), f"{what}: block {k} tile ({I}, {J}) should be empty"
+                    continue
+                e = np.linalg.norm(at - ot) / no
+                assert e <= bar, f"{what}: block {k} tile ({I}, {J}) relative error {e:.3e} > {bar}"
+
+
 @pytest.mark.parametrize("case", SIGMA_LAYERS, ids=lambda c: "-".join(str(v) for v in c))
 def test_layer_parity_at_discriminating_sigma(case):
     inp = _inputs(*case, sigma_q=pi.PARITY_SIGMA[case[3]])
@@ -137,6 +163,10 @@ def test_cnp_build_and_backward_parity(dtype, b, nblk, sigma):
     dqo = oracle.cnp_backward(q, b, dG.astype(np.float64))
     check(host64(G), Go, dtype, "G")
     check(host64(dq), dqo, dtype, "dq")
+    if dtype == "bf16":
+        # G rounded to bf16 alone leaves up to ~1.2% per tile of G - I at sigma 0.01
+        _tilewise(host64(G) - np.eye(b), Go - np.eye(b), "G - I", bar=5e-2)
+        _tilewise(_skew_from_packed(host64(dq), b), _skew_from_packed(dqo, b), "dq")
     # accumulate adds onto what is there
     px.poetx_cnp_backward(nblk, b, qd, torch.from_numpy(dG).cuda(), dq, 1, pd, ws, nb)
     torch.cuda.synchronize()
@@ -172,9 +202,12 @@ def test_cnp_full_batch_of_the_8b_block(sigma):
     assert np.array_equal(bits(sub_G), bits(G[147:150])) and np.array_equal(bits(sub_dq), bits(dq[147:150]))
     assert np.array_equal(bits(acc), bits(2 * dq))
     for t in [0, 1, 73, 74, 147, 148, 221, 295, 319]:
-        check(host64(G[t]), oracle.cnp_blocks(q[t:t + 1], b)[0], "bf16", f"G[{t}]")
-        check(host64(dq[t]), oracle.cnp_backward(q[t:t + 1], b, dG[t:t + 1].astype(np.float64))[0], "bf16",
-              f"dq[{t}]")
+        Go = oracle.cnp_blocks(q[t:t + 1], b)
+        dqo = oracle.cnp_backward(q[t:t + 1], b, dG[t:t + 1].astype(np.float64))
+        check(host64(G[t]), Go[0], "bf16", f"G[{t}]")
+        check(host64(dq[t]), dqo[0], "bf16", f"dq[{t}]")
+        _tilewise(host64(G[t:t + 1]) - np.eye(b), Go - np.eye(b), f"G[{t}] - I", bar=5e-2)
+        _tilewise(_skew_from_packed(host64(dq[t:t + 1]), b), _skew_from_packed(dqo, b), f"dq[{t}]")
 
 
 @pytest.mark.parametrize("name", ["block8b", "tiny"])
