@@ -287,18 +287,6 @@ __device__ __forceinline__ void box_row_bf16x32(uint32_t box, int r, int h, cons
                  : "memory");
   }
 }
-__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* p, const float* v) {
-  uint4* d = reinterpret_cast<uint4*>(p);
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    uint4 w;
-    w.x = pack_bf16x2(v[8 * u], v[8 * u + 1]);
-    w.y = pack_bf16x2(v[8 * u + 2], v[8 * u + 3]);
-    w.z = pack_bf16x2(v[8 * u + 4], v[8 * u + 5]);
-    w.w = pack_bf16x2(v[8 * u + 6], v[8 * u + 7]);
-    d[u] = w;
-  }
-}
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     cnp_pair_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmMN,
